@@ -1,0 +1,144 @@
+/*
+ * s2attn.h -- C ABI of the B200 (sm_100a) shifted-short-attention library.
+ *
+ * The operation (LongLoRA's S^2-Attn, as described on the LongLoRA pages):
+ *   - "LongLoRA paper notes" (smallflyingpig blog), section 3.3: a sequence of
+ *     length N is cut into groups of G tokens and attention runs only inside each
+ *     group, lowering the cost from O(N^2) to O(N^2 / (N/G)); a shifted pattern moves
+ *     the groups by half a group so that information crosses group borders
+ *     (drawing: groups 1-4, 5-8, 9-12 become 3-6, 7-10, 11-14).
+ *   - "LLaMA2 context to 100k" (nearauto.com), section on shift short attention:
+ *     two steps, (1) shift the tokens in half of the attention heads, (2) move the
+ *     features from the token dimension into the batch dimension.
+ *   - python88.com article, mechanism paragraph: the heads are split into two halves
+ *     and shifting one half lets neighbouring groups exchange information.
+ *   - "LongLoRA paper notes", section 3.1, and the model page (model.aibase.cn),
+ *     features list: inference uses ordinary full attention.
+ * Precisely, with scale = 1/sqrt(D) and shift s_h = G/2 for heads
+ * h >= H - shift_heads (0 otherwise): rolled row r of head h holds original token
+ * (r + s_h) mod N; group j owns rolled rows [jG, (j+1)G); query row r attends to the
+ * rolled rows r' of its own group with r' <= r (causal, in rolled order); the result
+ * of rolled row r is stored back at its original token.  G = N with shift_heads = 0
+ * is full causal attention (the inference case).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense row-major [B, N, H, D] ("token-major"); lse and delta are
+ *     [B, H, N] fp32, indexed by ORIGINAL token.
+ *   - Every pointer is a device pointer owned by the caller, 16-byte aligned; the
+ *     library never frees or keeps caller memory.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work and return; nothing synchronizes.
+ *   - Return value: S2ATTN_OK or a negative s2attn_status.  Argument errors are
+ *     detected on the host before anything is enqueued.  A failure inside a kernel
+ *     (a bounded wait that timed out) is recorded in a per-device error word that
+ *     s2attn_get_device_error() reads after the caller synchronizes.
+ *   - The calls are thread-safe with respect to each other.
+ */
+#ifndef S2ATTN_H_
+#define S2ATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  S2ATTN_OK = 0,
+  S2ATTN_ERR_INVALID_ARG = -1,    /* bad shape, null or misaligned pointer */
+  S2ATTN_ERR_UNSUPPORTED = -2,    /* valid, but not a shape this path handles */
+  S2ATTN_ERR_WORKSPACE = -3,      /* workspace missing or too small */
+  S2ATTN_ERR_CUDA = -4,           /* a CUDA runtime/driver call failed */
+  S2ATTN_ERR_DEVICE_TIMEOUT = -5  /* a kernel gave up on a bounded wait */
+} s2attn_status;
+
+/* Version of this ABI (major * 100 + minor). */
+int s2attn_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char* s2attn_status_string(int status);
+
+/*
+ * Forward pass, bf16 in / bf16 out, fp32 accumulation (tcgen05 tensor cores).
+ *   q, k, v : [B,N,H,D] bf16 inputs
+ *   o       : [B,N,H,D] bf16 output (attention output at each original token)
+ *   lse     : [B,H,N] fp32 output, natural log of sum over visible keys of exp(scale*q.k)
+ * Requirements: D == 128; G >= 1 divides N; 0 <= shift_heads <= H; G % 128 == 0;
+ * if shift_heads > 0 then (G/2) % 128 == 0.  Other valid shapes return
+ * S2ATTN_ERR_UNSUPPORTED (the fp32 entry points take any valid shape).
+ */
+int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N, int H, int D, int G,
+               int shift_heads, void* stream);
+
+/* Bytes of device workspace s2attn_bwd needs: an fp32 dQ accumulator [B,N,H,D]
+ * followed by delta [B,H,N] fp32 (each start 256-byte aligned).  0 on bad sizes. */
+size_t s2attn_bwd_workspace_bytes(int B, int N, int H, int D);
+
+/*
+ * Backward pass, bf16, same shape rules as s2attn_fwd.  Inputs: q, k, v, the
+ * forward output o and lse, and the output gradient dout.  Outputs dq, dk, dv
+ * ([B,N,H,D] bf16).  `workspace` (device, caller-owned, >= the size above,
+ * 256-byte aligned) is overwritten.  Runs s2attn_bwd_preprocess, s2attn_bwd_main
+ * and s2attn_bwd_dq_convert in that order on `stream`.
+ */
+int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+               void* dq, void* dk, void* dv, int B, int N, int H, int D, int G, int shift_heads, void* workspace,
+               size_t workspace_bytes, void* stream);
+
+/* Backward stage 1: delta[b,h,t] = sum_d dout[b,t,h,d] * o[b,t,h,d] (fp32, delta is
+ * [B,H,N]) and dq_acc ([B,N,H,D] fp32) := 0.  D must be 128. */
+int s2attn_bwd_preprocess(const void* o, const void* dout, float* delta, float* dq_acc, int B, int N, int H, int D,
+                          void* stream);
+
+/* Backward stage 2 (tensor cores): writes dk, dv (bf16) and adds the unscaled
+ * dQ = dS K into dq_acc (fp32, zeroed by stage 1).  Same shape rules as s2attn_fwd. */
+int s2attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                    const float* delta, float* dq_acc, void* dk, void* dv, int B, int N, int H, int D, int G,
+                    int shift_heads, void* stream);
+
+/* Backward stage 3: dq = bf16(dq_acc / sqrt(D)), round to nearest even. */
+int s2attn_bwd_dq_convert(const float* dq_acc, void* dq, int B, int N, int H, int D, void* stream);
+
+/*
+ * fp32 forward/backward on CUDA cores, any valid shape with 1 <= D <= 128
+ * (G >= 1 divides N; G even when shift_heads > 0).  Same tensor layouts, all fp32.
+ * s2attn_bwd_f32 uses the delta part of the workspace only
+ * (size from s2attn_bwd_workspace_bytes).
+ */
+int s2attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int N, int H, int D,
+                   int G, int shift_heads, void* stream);
+int s2attn_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* dout,
+                   const float* lse, float* dq, float* dk, float* dv, int B, int N, int H, int D, int G,
+                   int shift_heads, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * RoPE with position interpolation ("LongLoRA paper notes", section 3.4: positions
+ * [0, L) are squeezed into [0, L0)), applied in place to bf16 q and k ([B,N,H,D]).
+ * Token t is rotated as if at position t * pos_scale (pos_scale = L0 / N).  Element
+ * i < D/2 pairs with element i + D/2; the pair turns by angle a = (t*pos_scale) *
+ * theta_i with theta_i = base^(-2i/D).  Evaluation order (bit-for-bit contract):
+ *   theta_i = (float) pow(base, -2i/D) in double;  a = ((float)t * pos_scale) * theta_i
+ *   in float;  c, s = (float) cos/sin((double) a);  y1 = x1*c - x2*s;  y2 = x2*c + x1*s,
+ *   every product and sum rounded to fp32, then rounded to bf16 (nearest even).
+ * The cos/sin table is computed on the host on first use of each (device, N, D,
+ * pos_scale, base) and cached in device memory owned by the library until exit.
+ * Either q or k may be NULL.  Requires D % 16 == 0, D <= 256.
+ */
+int rope_pi_apply(void* q, void* k, int B, int N, int H, int D, float pos_scale, float base, void* stream);
+
+/*
+ * Reads the current device's error word: S2ATTN_OK if no kernel has failed since
+ * the last clear, else S2ATTN_ERR_DEVICE_TIMEOUT with *detail (if non-NULL) set to
+ * (kernel << 8) | site (kernel 1 = forward, 2 = backward).  Synchronize the streams
+ * that ran library kernels first.
+ */
+int s2attn_get_device_error(int* detail);
+
+/* Resets the current device's error word to 0 (synchronous). */
+int s2attn_clear_device_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S2ATTN_H_ */

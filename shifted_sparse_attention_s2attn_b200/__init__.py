@@ -1,1 +1,161 @@
+"""Python binding of the S^2-Attn C ABI (include/s2attn.h): argument marshalling only.
 
+Every function has the name of the C entry point it calls and takes torch tensors
+(device memory, contiguous [B,N,H,D]); shapes are read off the tensors, pointers and
+the current CUDA stream are passed through, and a non-zero status raises
+S2AttnError.  All arithmetic runs in the CUDA library libs2attn.so; if that library
+is missing, every call raises -- there is no fallback.
+"""
+import ctypes
+import os
+
+__all__ = [
+    "S2AttnError", "capi", "library_path",
+    "s2attn_fwd", "s2attn_bwd", "s2attn_bwd_workspace_bytes", "s2attn_bwd_preprocess", "s2attn_bwd_main",
+    "s2attn_bwd_dq_convert", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply",
+    "get_device_error", "clear_device_error",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libs2attn.so")
+
+STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "workspace", -4: "CUDA error",
+          -5: "device timeout"}
+
+
+class S2AttnError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} failed: status {status} ({STATUS.get(status, 'unknown')})")
+        self.status = status
+
+
+_lib = None
+
+
+def capi():
+    """The loaded C library (ctypes), with argument types declared."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError(f"CUDA library not built: {library_path} is missing "
+                           "(run: python -m shifted_sparse_attention_s2attn_b200._build)")
+    lib = ctypes.CDLL(library_path)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "s2attn_version": ([], I),
+        "s2attn_status_string": ([I], ctypes.c_char_p),
+        "s2attn_fwd": ([P, P, P, P, P, I, I, I, I, I, I, P], I),
+        "s2attn_bwd_workspace_bytes": ([I, I, I, I], Z),
+        "s2attn_bwd": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, Z, P], I),
+        "s2attn_bwd_preprocess": ([P, P, P, P, I, I, I, I, P], I),
+        "s2attn_bwd_main": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P], I),
+        "s2attn_bwd_dq_convert": ([P, P, I, I, I, I, P], I),
+        "s2attn_fwd_f32": ([P, P, P, P, P, I, I, I, I, I, I, P], I),
+        "s2attn_bwd_f32": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, Z, P], I),
+        "rope_pi_apply": ([P, P, I, I, I, I, F, F, P], I),
+        "s2attn_get_device_error": ([ctypes.POINTER(I)], I),
+        "s2attn_clear_device_error": ([], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise S2AttnError(fn, rc)
+
+
+def _bnhd(t, name):
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B,N,H,D] tensor")
+    return tuple(t.shape)
+
+
+def s2attn_fwd(q, k, v, o, lse, G, shift_heads, stream=None):
+    """bf16 forward: o <- S^2-Attn(q, k, v), lse <- [B,H,N] fp32 log-sum-exp."""
+    B, N, H, D = _bnhd(q, "q")
+    _check("s2attn_fwd", capi().s2attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, N, H, D, G,
+                                           shift_heads, _stream(stream)))
+
+
+def s2attn_bwd_workspace_bytes(B, N, H, D):
+    return int(capi().s2attn_bwd_workspace_bytes(B, N, H, D))
+
+
+def s2attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, workspace, stream=None):
+    """bf16 backward into dq, dk, dv.  workspace: a uint8 device tensor of at least
+    s2attn_bwd_workspace_bytes(B,N,H,D) bytes, 256-byte aligned."""
+    B, N, H, D = _bnhd(q, "q")
+    _check("s2attn_bwd", capi().s2attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                                           _ptr(dk), _ptr(dv), B, N, H, D, G, shift_heads, _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def s2attn_bwd_preprocess(o, dout, delta, dq_acc, stream=None):
+    B, N, H, D = _bnhd(o, "o")
+    _check("s2attn_bwd_preprocess", capi().s2attn_bwd_preprocess(_ptr(o), _ptr(dout), _ptr(delta), _ptr(dq_acc),
+                                                                 B, N, H, D, _stream(stream)))
+
+
+def s2attn_bwd_main(q, k, v, dout, lse, delta, dq_acc, dk, dv, G, shift_heads, stream=None):
+    B, N, H, D = _bnhd(q, "q")
+    _check("s2attn_bwd_main", capi().s2attn_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(delta),
+                                                     _ptr(dq_acc), _ptr(dk), _ptr(dv), B, N, H, D, G, shift_heads,
+                                                     _stream(stream)))
+
+
+def s2attn_bwd_dq_convert(dq_acc, dq, stream=None):
+    B, N, H, D = _bnhd(dq, "dq")
+    _check("s2attn_bwd_dq_convert", capi().s2attn_bwd_dq_convert(_ptr(dq_acc), _ptr(dq), B, N, H, D,
+                                                                 _stream(stream)))
+
+
+def s2attn_fwd_f32(q, k, v, o, lse, G, shift_heads, stream=None):
+    B, N, H, D = _bnhd(q, "q")
+    _check("s2attn_fwd_f32", capi().s2attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, N, H, D, G,
+                                                   shift_heads, _stream(stream)))
+
+
+def s2attn_bwd_f32(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, workspace, stream=None):
+    B, N, H, D = _bnhd(q, "q")
+    _check("s2attn_bwd_f32", capi().s2attn_bwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                                   _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, D, G, shift_heads,
+                                                   _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                   _stream(stream)))
+
+
+def rope_pi_apply(q, k, pos_scale, base=10000.0, stream=None):
+    """In-place RoPE with position interpolation on bf16 q and/or k ([B,N,H,D])."""
+    ref = q if q is not None else k
+    B, N, H, D = _bnhd(ref, "q/k")
+    _check("rope_pi_apply", capi().rope_pi_apply(_ptr(q), _ptr(k), B, N, H, D, float(pos_scale), float(base),
+                                                 _stream(stream)))
+
+
+def get_device_error():
+    """(status, detail) of the current device's error word; synchronize first."""
+    d = ctypes.c_int(0)
+    rc = capi().s2attn_get_device_error(ctypes.byref(d))
+    return rc, d.value
+
+
+def clear_device_error():
+    _check("s2attn_clear_device_error", capi().s2attn_clear_device_error())

@@ -1,0 +1,47 @@
+// s2_internal.h -- launch functions shared between the library's translation units.
+// Host-only declarations; kernels live in the .cu files that define these.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace s2 {
+
+// Device error codes (first failure wins; read with s2attn_get_device_error).
+// code = (kernel << 8) | site
+enum Kernel : int { K_FWD = 1, K_BWD = 2 };
+
+// Problem description after validation.  Rows of a [B,N,H,D] tensor for head h
+// are addressed through 3-D tensor maps with dims {D, H, B*N}.
+struct Shape {
+  int B, N, H, D, G, shift_heads;
+};
+
+// Forward, bf16, D == 128: one launch of the tcgen05 kernel.
+cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             void* o, float* lse, const Shape& s, int* err, cudaStream_t st);
+
+// Backward main kernel, bf16, D == 128: dK, dV written, dQ accumulated (fp32) into dq_acc.
+cudaError_t launch_bwd_sm100(const CUtensorMap& tq64, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tdo64, const CUtensorMap& tdq_acc, const float* lse,
+                             const float* delta, void* dk, void* dv, const Shape& s, int* err, cudaStream_t st);
+
+// delta[b,h,t] = sum_d dO*O (fp32) and dq_acc := 0.
+cudaError_t launch_bwd_preprocess(const void* o, const void* dout, float* delta, float* dq_acc, const Shape& s,
+                                  cudaStream_t st);
+// dq = bf16(scale * dq_acc)
+cudaError_t launch_dq_convert(const float* dq_acc, void* dq, const Shape& s, cudaStream_t st);
+
+// fp32 CUDA-core path (any valid shape).
+cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, const Shape& s,
+                           cudaStream_t st);
+cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* dout,
+                           const float* lse, float* dq, float* dk, float* dv, float* delta, const Shape& s,
+                           cudaStream_t st);
+
+// RoPE-PI in place on bf16 q and k, with a cos/sin table [N, D/2] (fp32 each).
+cudaError_t launch_rope_pi(void* q, void* k, const float* cos_tab, const float* sin_tab, int B, int N, int H,
+                           int D, cudaStream_t st);
+
+}  // namespace s2

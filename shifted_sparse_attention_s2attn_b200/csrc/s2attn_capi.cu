@@ -1,0 +1,308 @@
+// s2attn_capi.cu -- the extern "C" boundary: argument validation, tensor-map
+// construction, the RoPE table cache, the device error word, and kernel launches.
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "s2_internal.h"
+#include "s2attn.h"
+
+namespace {
+
+__device__ int g_error_word;
+
+constexpr int kMaxDevices = 64;
+
+// ---- error word -----------------------------------------------------------------
+int* error_word_ptr() {
+  static std::mutex mu;
+  static int* cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+// ---- tensor maps ----------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// A [B,N,H,D] tensor viewed as 3-D {D, H, B*N}; a box is box_rows tokens x box_cols
+// elements of one head.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, size_t esize, int B, int N, int H, int D,
+              uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)B * (cuuint64_t)N};
+  cuuint64_t strides[2] = {(cuuint64_t)D * esize, (cuuint64_t)H * D * esize};
+  cuuint32_t box[3] = {box_cols, 1, box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool map_bf16_sw128(CUtensorMap* m, const void* base, const s2::Shape& s, uint32_t rows) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, s.B, s.N, s.H, s.D, 64, rows,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// ---- validation -----------------------------------------------------------------
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int N, int H, int D, int G, int shift_heads) {
+  if (B < 1 || N < 1 || H < 1 || D < 1 || G < 1) return S2ATTN_ERR_INVALID_ARG;
+  if (N % G != 0) return S2ATTN_ERR_INVALID_ARG;
+  if (shift_heads < 0 || shift_heads > H) return S2ATTN_ERR_INVALID_ARG;
+  if (shift_heads > 0 && (G % 2) != 0) return S2ATTN_ERR_INVALID_ARG;
+  if ((long long)B * N > INT_MAX / 2) return S2ATTN_ERR_INVALID_ARG;
+  if ((long long)B * N * H > (LLONG_MAX / 8) / D) return S2ATTN_ERR_INVALID_ARG;
+  return S2ATTN_OK;
+}
+
+int check_tensor_core_shape(int B, int N, int H, int D, int G, int shift_heads) {
+  int rc = check_shape(B, N, H, D, G, shift_heads);
+  if (rc) return rc;
+  if (D != 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (G % 128 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if (shift_heads > 0 && (G / 2) % 128 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * H * (N / G) * (G / 128) > INT_MAX) return S2ATTN_ERR_UNSUPPORTED;
+  return S2ATTN_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? S2ATTN_OK : S2ATTN_ERR_CUDA; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---- RoPE tables ------------------------------------------------------------------
+struct RopeTable {
+  float* cos_d = nullptr;
+  float* sin_d = nullptr;
+};
+
+// theta_i = (float) base^(-2i/D) (pow in double); a = ((float)t * pos_scale) * theta_i in
+// float; table entries (float) cos((double)a), (float) sin((double)a).
+int rope_table(int dev, int N, int D, float pos_scale, float base, RopeTable* out) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, uint32_t, uint32_t>, RopeTable> cache;
+  uint32_t ps, bs;
+  std::memcpy(&ps, &pos_scale, 4);
+  std::memcpy(&bs, &base, 4);
+  auto key = std::make_tuple(dev, N, D, ps, bs);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *out = it->second;
+    return S2ATTN_OK;
+  }
+  const int half = D / 2;
+  std::vector<float> c((size_t)N * half), s((size_t)N * half);
+  std::vector<float> theta(half);
+  for (int i = 0; i < half; ++i) theta[i] = (float)std::pow((double)base, -2.0 * (double)i / (double)D);
+  for (int t = 0; t < N; ++t) {
+    volatile float pos = (float)t * pos_scale;
+    for (int i = 0; i < half; ++i) {
+      volatile float a = pos * theta[i];
+      c[(size_t)t * half + i] = (float)std::cos((double)a);
+      s[(size_t)t * half + i] = (float)std::sin((double)a);
+    }
+  }
+  RopeTable tab;
+  const size_t bytes = sizeof(float) * c.size();
+  if (cudaMalloc(&tab.cos_d, bytes) != cudaSuccess) return S2ATTN_ERR_CUDA;
+  if (cudaMalloc(&tab.sin_d, bytes) != cudaSuccess) {
+    cudaFree(tab.cos_d);
+    return S2ATTN_ERR_CUDA;
+  }
+  if (cudaMemcpy(tab.cos_d, c.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(tab.sin_d, s.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(tab.cos_d);
+    cudaFree(tab.sin_d);
+    return S2ATTN_ERR_CUDA;
+  }
+  cache[key] = tab;
+  *out = tab;
+  return S2ATTN_OK;
+}
+
+int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                  const float* delta, float* dq_acc, void* dk, void* dv, const s2::Shape& s, cudaStream_t st) {
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  if (!map_bf16_sw128(&tq, q, s, 64) || !map_bf16_sw128(&tk, k, s, 128) || !map_bf16_sw128(&tv, v, s, 128) ||
+      !map_bf16_sw128(&tdo, dout, s, 64) ||
+      !make_map(&tdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, s.B, s.N, s.H, s.D, 128, 64,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return S2ATTN_ERR_CUDA;
+  int* err = error_word_ptr();
+  if (!err) return S2ATTN_ERR_CUDA;
+  return cuda_status(s2::launch_bwd_sm100(tq, tk, tv, tdo, tdq, lse, delta, dk, dv, s, err, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int s2attn_version(void) { return 100; }
+
+const char* s2attn_status_string(int status) {
+  switch (status) {
+    case S2ATTN_OK: return "ok";
+    case S2ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case S2ATTN_ERR_UNSUPPORTED: return "unsupported shape for this path";
+    case S2ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case S2ATTN_ERR_CUDA: return "CUDA call failed";
+    case S2ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N, int H, int D, int G,
+               int shift_heads, void* stream) {
+  int rc = check_tensor_core_shape(B, N, H, D, G, shift_heads);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return S2ATTN_ERR_INVALID_ARG;
+  const s2::Shape s{B, N, H, D, G, shift_heads};
+  CUtensorMap tq, tk, tv;
+  if (!map_bf16_sw128(&tq, q, s, 128) || !map_bf16_sw128(&tk, k, s, 128) || !map_bf16_sw128(&tv, v, s, 128))
+    return S2ATTN_ERR_CUDA;
+  int* err = error_word_ptr();
+  if (!err) return S2ATTN_ERR_CUDA;
+  return cuda_status(s2::launch_fwd_sm100(tq, tk, tv, o, lse, s, err, static_cast<cudaStream_t>(stream)));
+}
+
+size_t s2attn_bwd_workspace_bytes(int B, int N, int H, int D) {
+  if (B < 1 || N < 1 || H < 1 || D < 1) return 0;
+  return align256((size_t)B * N * H * D * sizeof(float)) + align256((size_t)B * H * N * sizeof(float));
+}
+
+int s2attn_bwd_preprocess(const void* o, const void* dout, float* delta, float* dq_acc, int B, int N, int H, int D,
+                          void* stream) {
+  int rc = check_shape(B, N, H, D, N, 0);
+  if (rc) return rc;
+  if (D != 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(o) || !aligned16(dout) || !aligned16(delta) || !aligned16(dq_acc)) return S2ATTN_ERR_INVALID_ARG;
+  const s2::Shape s{B, N, H, D, N, 0};
+  return cuda_status(s2::launch_bwd_preprocess(o, dout, delta, dq_acc, s, static_cast<cudaStream_t>(stream)));
+}
+
+int s2attn_bwd_main(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                    const float* delta, float* dq_acc, void* dk, void* dv, int B, int N, int H, int D, int G,
+                    int shift_heads, void* stream) {
+  int rc = check_tensor_core_shape(B, N, H, D, G, shift_heads);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(delta) || !aligned16(dq_acc) || !aligned16(dk) || !aligned16(dv))
+    return S2ATTN_ERR_INVALID_ARG;
+  const s2::Shape s{B, N, H, D, G, shift_heads};
+  return bwd_main_impl(q, k, v, dout, lse, delta, dq_acc, dk, dv, s, static_cast<cudaStream_t>(stream));
+}
+
+int s2attn_bwd_dq_convert(const float* dq_acc, void* dq, int B, int N, int H, int D, void* stream) {
+  int rc = check_shape(B, N, H, D, N, 0);
+  if (rc) return rc;
+  if (D % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(dq_acc) || !aligned16(dq)) return S2ATTN_ERR_INVALID_ARG;
+  const s2::Shape s{B, N, H, D, N, 0};
+  return cuda_status(s2::launch_dq_convert(dq_acc, dq, s, static_cast<cudaStream_t>(stream)));
+}
+
+int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+               void* dq, void* dk, void* dv, int B, int N, int H, int D, int G, int shift_heads, void* workspace,
+               size_t workspace_bytes, void* stream) {
+  int rc = check_tensor_core_shape(B, N, H, D, G, shift_heads);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return S2ATTN_ERR_INVALID_ARG;
+  const size_t need = s2attn_bwd_workspace_bytes(B, N, H, D);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return S2ATTN_ERR_WORKSPACE;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256((size_t)B * N * H * D * 4));
+  const s2::Shape s{B, N, H, D, G, shift_heads};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = cuda_status(s2::launch_bwd_preprocess(o, dout, delta, dq_acc, s, st)))) return rc;
+  if ((rc = bwd_main_impl(q, k, v, dout, lse, delta, dq_acc, dk, dv, s, st))) return rc;
+  return cuda_status(s2::launch_dq_convert(dq_acc, dq, s, st));
+}
+
+int s2attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int N, int H, int D,
+                   int G, int shift_heads, void* stream) {
+  int rc = check_shape(B, N, H, D, G, shift_heads);
+  if (rc) return rc;
+  if (D > 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return S2ATTN_ERR_INVALID_ARG;
+  const s2::Shape s{B, N, H, D, G, shift_heads};
+  return cuda_status(s2::launch_fwd_f32(q, k, v, o, lse, s, static_cast<cudaStream_t>(stream)));
+}
+
+int s2attn_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* dout,
+                   const float* lse, float* dq, float* dk, float* dv, int B, int N, int H, int D, int G,
+                   int shift_heads, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_shape(B, N, H, D, G, shift_heads);
+  if (rc) return rc;
+  if (D > 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return S2ATTN_ERR_INVALID_ARG;
+  const size_t need = s2attn_bwd_workspace_bytes(B, N, H, D);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return S2ATTN_ERR_WORKSPACE;
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256((size_t)B * N * H * D * 4));
+  const s2::Shape s{B, N, H, D, G, shift_heads};
+  return cuda_status(
+      s2::launch_bwd_f32(q, k, v, o, dout, lse, dq, dk, dv, delta, s, static_cast<cudaStream_t>(stream)));
+}
+
+int rope_pi_apply(void* q, void* k, int B, int N, int H, int D, float pos_scale, float base, void* stream) {
+  if (B < 1 || N < 1 || H < 1 || D < 16 || D % 16 != 0 || D > 256) return S2ATTN_ERR_INVALID_ARG;
+  if ((long long)B * N * H > (LLONG_MAX / 8) / D) return S2ATTN_ERR_INVALID_ARG;
+  if (!q && !k) return S2ATTN_ERR_INVALID_ARG;
+  if ((q && !aligned16(q)) || (k && !aligned16(k))) return S2ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(pos_scale) || !std::isfinite(base) || !(base > 0.f)) return S2ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return S2ATTN_ERR_CUDA;
+  RopeTable tab;
+  int rc = rope_table(dev, N, D, pos_scale, base, &tab);
+  if (rc) return rc;
+  return cuda_status(
+      s2::launch_rope_pi(q, k, tab.cos_d, tab.sin_d, B, N, H, D, static_cast<cudaStream_t>(stream)));
+}
+
+int s2attn_get_device_error(int* detail) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof(int)) != cudaSuccess) return S2ATTN_ERR_CUDA;
+  if (detail) *detail = v;
+  return v == 0 ? S2ATTN_OK : S2ATTN_ERR_DEVICE_TIMEOUT;
+}
+
+int s2attn_clear_device_error(void) {
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) == cudaSuccess ? S2ATTN_OK : S2ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,366 @@
+// s2attn_fwd_sm100.cu -- S^2-Attn forward on B200 (sm_100a): tcgen05 MMAs with
+// TMEM accumulators, TMA tile loads, warp-specialised CTA.
+//
+// Method (LongLoRA pages: "LongLoRA paper notes" section 3.3; nearauto.com article,
+// "shift short attention" steps (1) and (2)): for every head, cut the sequence into
+// groups of G tokens and run causal softmax attention inside each group; heads
+// h >= H - shift_heads first see the sequence rolled by G/2.  Here the roll and the
+// token->batch regrouping are pure address arithmetic: rolled row r of a shifted
+// head is original token (r + G/2) mod N, and because G/2 and N are multiples of the
+// 128-row tile, every 128-row tile of rolled rows is a contiguous run of original
+// rows.  Each TMA box therefore loads straight from the original [B,N,H,D] tensor
+// and each output row is stored straight back to its original token: no rolled copy
+// of Q/K/V/O ever exists.
+//
+// CTA work item: (batch b, head h, group j, pair m) -> the two query tiles 2m and
+// 2m+1 of the group (128 rows each), which share every K/V tile they load.  Only the
+// causal lower triangle is visited: query tile qt needs key tiles 0..qt, and only
+// tile qt (the diagonal) is masked.  Items are ordered heaviest first.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax for query tile 0 (thread = row; TMEM lanes 0..127)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer (Q once; K and V through 2-stage rings); TMEM owner
+//   warp  9    MMA issuer: S_i = Q_i K^T (SS), O_i += P_i V (TS: P read from TMEM)
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512); P_i is
+// written as bf16 pairs over the first 64 columns of S_i.  tcgen05 MMAs issued by
+// one thread execute in issue order, so S_i(t+1) may be issued right after the
+// PV_i(t) that still reads P_i(t) from the same columns.
+//
+// Softmax: online, base 2, with a lazy rescale -- the running max is only moved (and
+// O rescaled) when a row's max grows by more than 2^8, so P <= 256 and most tiles
+// skip the O round trip through registers.
+#include "s2_internal.h"
+#include "s2_ptx.cuh"
+
+namespace s2 {
+namespace fwd {
+
+constexpr int BM = 128;                      // query rows per tile
+constexpr int BN = 128;                      // keys per tile
+constexpr int HD = 128;                      // head dim
+constexpr int NBOX = HD / 64;                // 64-column (128-byte) swizzle boxes per row
+constexpr uint32_t BOX_BYTES = 128 * 128;    // 128 rows x 128 B
+constexpr uint32_t TILE_BYTES = NBOX * BOX_BYTES;
+constexpr int STAGES = 2;
+constexpr int NTHREADS = 320;
+constexpr int WARP_LOAD = 8, WARP_MMA = 9;
+
+constexpr uint32_t OFF_Q0 = 0;
+constexpr uint32_t OFF_Q1 = OFF_Q0 + TILE_BYTES;
+constexpr uint32_t OFF_K = OFF_Q1 + TILE_BYTES;
+constexpr uint32_t OFF_V = OFF_K + STAGES * TILE_BYTES;
+constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE_BYTES;
+// barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_ready[2], o_final[2], drain
+constexpr int NBARS = 16;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
+
+// TMEM column of S_i / O_i for query tile i
+__device__ __forceinline__ uint32_t tm_s(int i) { return i == 0 ? 0u : 128u; }
+__device__ __forceinline__ uint32_t tm_o(int i) { return i == 0 ? 256u : 384u; }
+constexpr float LN2 = 0.69314718055994530942f;
+
+struct Params {
+  __nv_bfloat16* o;
+  float* lse;
+  int B, N, H, G, shift_heads;
+  int n_qt, n_pairs, n_groups;
+  float sl2;  // softmax scale * log2(e)
+  int* err;
+};
+
+enum Site : int { SITE_LOAD = 1, SITE_MMA = 2, SITE_SOFTMAX = 3, SITE_EPILOGUE = 4, SITE_DRAIN = 5 };
+
+__device__ __forceinline__ void issue_s(uint32_t d, uint32_t sq, uint32_t sk, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk) {
+    const uint32_t off = (kk / 4) * BOX_BYTES + (kk % 4) * 32;
+    mma_ss(d, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ void issue_pv(uint32_t d, uint32_t tp, uint32_t sv, uint32_t idesc, bool first) {
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk) {
+    // B = V^T viewed MN-major: 16 key rows (2 KB) per k-step, 64-column boxes BOX_BYTES apart.
+    mma_ts(d, tp + kk * 8, sdesc_sw128(sv + kk * 2048, BOX_BYTES, 1024), idesc, (first && kk == 0) ? 0u : 1u);
+  }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    s2attn_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                      const __grid_constant__ CUtensorMap tv, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 3;
+  uint64_t* v_full = bars + 5;
+  uint64_t* v_empty = bars + 7;
+  uint64_t* s_full = bars + 9;
+  uint64_t* p_ready = bars + 11;
+  uint64_t* o_final = bars + 13;
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // ---- work item -------------------------------------------------------------
+  const int per_m = p.B * p.H * p.n_groups;
+  const int m = p.n_pairs - 1 - (int)(blockIdx.x / per_m);
+  int rest = (int)(blockIdx.x % per_m);
+  const int j = rest % p.n_groups;
+  rest /= p.n_groups;
+  const int h = rest % p.H;
+  const int b = rest / p.H;
+  const int qa = 2 * m, qb = 2 * m + 1;
+  const bool has_b = qb < p.n_qt;
+  const int nkv = (has_b ? qb : qa) + 1;
+  const int shift = (h >= p.H - p.shift_heads) ? p.G / 2 : 0;
+  const int group_row0 = j * p.G;
+  // first original token of the 128-row tile `tile` of this group (tiles never wrap)
+  auto tile_token0 = [&](int tile) {
+    int t = group_row0 + tile * BM + shift;
+    return t >= p.N ? t - p.N : t;
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_ready[i], 4);
+      mbar_init(&o_final[i], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = (*(volatile int*)p.err != 0) ? 1 : 0;  // an earlier CTA failed: skip the work
+    fence_mbar_init();
+  }
+  if (warp == WARP_LOAD) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = *abort_flag != 0;
+
+  if (!skip && warp == WARP_LOAD && lane == 0) {
+    // ---------------- TMA producer ----------------
+    prefetch_tmap(&tq);
+    prefetch_tmap(&tk);
+    prefetch_tmap(&tv);
+    bool ok = true;
+    const int row_base = b * p.N;
+    mbar_arrive_expect_tx(q_full, (has_b ? 2u : 1u) * TILE_BYTES);
+    for (int x = 0; x < NBOX; ++x) {
+      tma_load_3d(smem + OFF_Q0 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(qa), q_full);
+      if (has_b) tma_load_3d(smem + OFF_Q1 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(qb), q_full);
+    }
+    int armed = 0;  // K/V tiles issued
+    for (int t = 0; t < nkv && ok; ++t) {
+      const int st = t % STAGES;
+      const uint32_t ph = (t / STAGES) & 1;
+      const int row = row_base + tile_token0(t);
+      ok = wait_bounded(&k_empty[st], ph ^ 1, abort_flag, p.err);
+      if (!ok) break;
+      mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
+      for (int x = 0; x < NBOX; ++x) tma_load_3d(smem + OFF_K + st * TILE_BYTES + x * BOX_BYTES, &tk, x * 64, h, row, &k_full[st]);
+      ok = wait_bounded(&v_empty[st], ph ^ 1, abort_flag, p.err);
+      if (!ok) {
+        armed = -(t + 1);  // K of tile t in flight, V not
+        break;
+      }
+      mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
+      for (int x = 0; x < NBOX; ++x) tma_load_3d(smem + OFF_V + st * TILE_BYTES + x * BOX_BYTES, &tv, x * 64, h, row, &v_full[st]);
+      armed = t + 1;
+    }
+    if (!ok) {
+      report_error(p.err, (K_FWD << 8) | SITE_LOAD);
+      *abort_flag = 1;
+    }
+    // Drain: every copy this thread started must land before the CTA can exit.
+    bool dok = wait_drain(q_full, 0);
+    const int nk = armed >= 0 ? armed : -armed, nv = armed >= 0 ? armed : -armed - 1;
+    for (int t = (nk > STAGES ? nk - STAGES : 0); t < nk; ++t) dok &= wait_drain(&k_full[t % STAGES], (t / STAGES) & 1);
+    for (int t = (nv > STAGES ? nv - STAGES : 0); t < nv; ++t) dok &= wait_drain(&v_full[t % STAGES], (t / STAGES) & 1);
+    if (!dok) report_error(p.err, (K_FWD << 8) | SITE_DRAIN);
+  } else if (!skip && warp == WARP_MMA && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    const uint32_t id_s = idesc_bf16_f32(BM, BN, false, false);
+    const uint32_t id_pv = idesc_bf16_f32(BM, HD, false, true);
+    const uint32_t sq[2] = {smem_u32(smem + OFF_Q0), smem_u32(smem + OFF_Q1)};
+    const uint32_t sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
+    const int qts[2] = {qa, qb};
+    uint32_t p_phase[2] = {0, 0};
+    bool ok = wait_bounded(q_full, 0, abort_flag, p.err);
+    for (int t = 0; t <= nkv && ok; ++t) {
+      const bool has_prev = t > 0, has_cur = t < nkv;
+      if (has_cur) ok = wait_bounded(&k_full[t % STAGES], (t / STAGES) & 1, abort_flag, p.err);
+      if (ok && has_prev) ok = wait_bounded(&v_full[(t - 1) % STAGES], ((t - 1) / STAGES) & 1, abort_flag, p.err);
+      if (!ok) break;
+      tc_fence_after();
+      for (int i = 0; i < 2 && ok; ++i) {
+        if (i == 1 && !has_b) break;
+        const int qt = qts[i];
+        if (has_prev && t - 1 <= qt) {
+          ok = wait_bounded(&p_ready[i], p_phase[i], abort_flag, p.err);
+          p_phase[i] ^= 1;
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(tmem + tm_o(i), tmem + tm_s(i), sv + ((t - 1) % STAGES) * TILE_BYTES, id_pv, t - 1 == 0);
+          if (t - 1 == qt) mma_commit(&o_final[i]);
+        }
+        if (has_cur && t <= qt) {
+          issue_s(tmem + tm_s(i), sq[i], sk + (t % STAGES) * TILE_BYTES, id_s);
+          mma_commit(&s_full[i]);
+        }
+      }
+      if (!ok) break;
+      if (has_prev) mma_commit(&v_empty[(t - 1) % STAGES]);
+      if (has_cur) mma_commit(&k_empty[t % STAGES]);
+    }
+    if (!ok) {
+      report_error(p.err, (K_FWD << 8) | SITE_MMA);
+      *abort_flag = 1;
+    }
+    // Drain: all issued MMAs complete before TMEM is released.
+    mma_commit(drain);
+    if (!wait_drain(drain, 0)) report_error(p.err, (K_FWD << 8) | SITE_DRAIN);
+  } else if (!skip && warp < 8) {
+    // ---------------- softmax warpgroups ----------------
+    const int i = warp / 4;
+    if (i == 0 || has_b) {
+      const int qt = i == 0 ? qa : qb;
+      const int row = (warp % 4) * 32 + lane;
+      const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
+      const uint32_t t_s = lane_addr + tm_s(i), t_o = lane_addr + tm_o(i);
+      const float sl2 = p.sl2;
+      float m_run = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      for (int t = 0; t <= qt; ++t) {
+        ok = wait_bounded(&s_full[i], t & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t s0[64], s1[64];
+        tmem_ld_x64(t_s, s0);
+        tmem_ld_x64(t_s + 64, s1);
+        float x[128];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          x[c] = __uint_as_float(s0[c]) * sl2;
+          x[c + 64] = __uint_as_float(s1[c]) * sl2;
+        }
+        if (t == qt) {  // diagonal tile: key column c is visible to row `row` iff c <= row
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > row) x[c] = -INFINITY;
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+        const float m_new = fmaxf(m_run, mx);
+        const bool need = (m_new - m_run) > 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
+          if (need) m_run = m_new;
+          l_run *= alpha;
+          if (t > 0) {
+            // O_i was last written by PV_i(t-1), which completed before S_i(t) did.
+#pragma unroll
+            for (int c = 0; c < HD; c += 32) {
+              uint32_t r[32];
+              tmem_ld_x32(t_o + c, r);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              tmem_st_x32(t_o + c, r);
+            }
+          }
+        }
+        float sum = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float p0 = ex2_approx(x[2 * c] - m_run);
+          const float p1 = ex2_approx(x[2 * c + 1] - m_run);
+          sum += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        l_run += sum;
+        tmem_st_x64(t_s, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready[i]);
+      }
+      if (ok) ok = wait_bounded(&o_final[i], 0, abort_flag, p.err);
+      if (!ok) {
+        report_error(p.err, (K_FWD << 8) | SITE_SOFTMAX);
+        *abort_flag = 1;
+      } else {
+        // ---- epilogue: O row / l, stored at its original token; lse in natural log ----
+        tc_fence_after();
+        const int tok = tile_token0(qt) + row;
+        const float inv_l = 1.0f / l_run;
+        __nv_bfloat16* orow = p.o + ((size_t)(b * p.N + tok) * p.H + h) * HD;
+#pragma unroll
+        for (int c = 0; c < HD; c += 32) {
+          uint32_t r[32];
+          tmem_ld_x32(t_o + c, r);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+        p.lse[((size_t)b * p.H + h) * p.N + tok] = (m_run + log2f(l_run)) * LN2;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_LOAD) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fwd
+
+cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                             float* lse, const Shape& s, int* err, cudaStream_t st) {
+  fwd::Params p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = s.B;
+  p.N = s.N;
+  p.H = s.H;
+  p.G = s.G;
+  p.shift_heads = s.shift_heads;
+  p.n_qt = s.G / fwd::BM;
+  p.n_pairs = (p.n_qt + 1) / 2;
+  p.n_groups = s.N / s.G;
+  p.sl2 = (float)(1.4426950408889634 / sqrt((double)s.D));
+  p.err = err;
+  const long long grid = (long long)p.n_pairs * s.B * s.H * p.n_groups;
+  if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(fwd::s2attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)fwd::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  fwd::s2attn_fwd_kernel<<<(unsigned)grid, fwd::NTHREADS, fwd::SMEM_BYTES, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace s2

@@ -1,0 +1,101 @@
+"""CPU-only checks of the C ABI: the library builds for sm_100a, loads, exports every
+function include/s2attn.h declares, and rejects bad arguments on the host (these
+calls return before any CUDA work, so no GPU is needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from shifted_sparse_attention_s2attn_b200 import _build, capi
+    _build.build()
+    return capi()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "s2attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|const char\s*\*|void)\s*\*?\s*"
+                                 r"([a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("s2attn_fwd", "s2attn_bwd", "rope_pi_apply", "s2attn_bwd_workspace_bytes",
+                     "s2attn_fwd_f32", "s2attn_bwd_f32", "s2attn_get_device_error"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.s2attn_version() == 100
+    assert lib.s2attn_status_string(0) == b"ok"
+    assert lib.s2attn_status_string(-2).startswith(b"unsupported")
+
+
+def test_workspace_size(lib):
+    B, N, H, D = 1, 32768, 32, 128
+    acc = B * N * H * D * 4
+    delta = B * H * N * 4
+    assert lib.s2attn_bwd_workspace_bytes(B, N, H, D) == acc + delta
+    assert lib.s2attn_bwd_workspace_bytes(0, N, H, D) == 0
+
+
+NULL = None
+
+
+@pytest.mark.parametrize("args,status", [
+    ((1, 1000, 2, 128, 300, 0), -1),    # G does not divide N
+    ((1, 1024, 2, 128, 512, 3), -1),    # more shifted heads than heads
+    ((1, 1024, 2, 128, 0, 0), -1),      # G = 0
+    ((0, 1024, 2, 128, 512, 0), -1),    # empty batch
+    ((1, 0, 2, 128, 512, 0), -1),       # empty sequence
+    ((1, 1024, 2, 64, 512, 0), -2),     # D = 64: fp32 path only
+    ((1, 768, 2, 128, 384, 1), -2),     # G/2 not a multiple of the 128-row tile
+    ((1, 960, 2, 128, 320, 0), -2),     # G not a multiple of 128
+    ((1, 1024, 2, 128, 512, 1), -1),    # valid shape, null pointers
+])
+def test_fwd_bwd_validation(lib, args, status):
+    assert lib.s2attn_fwd(NULL, NULL, NULL, NULL, NULL, *args, NULL) == status
+    assert lib.s2attn_bwd(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, *args, NULL, 0, NULL) == status
+
+
+def test_misaligned_pointer_rejected(lib):
+    p = ctypes.c_void_p(0x1000 + 8)
+    assert lib.s2attn_fwd(p, p, p, p, p, 1, 1024, 2, 128, 512, 0, NULL) == -1
+
+
+def test_f32_validation(lib):
+    assert lib.s2attn_fwd_f32(NULL, NULL, NULL, NULL, NULL, 1, 90, 3, 40, 18, 1, NULL) == -1   # null pointers
+    assert lib.s2attn_fwd_f32(NULL, NULL, NULL, NULL, NULL, 1, 90, 3, 40, 9, 1, NULL) == -1    # odd G shifted
+    assert lib.s2attn_fwd_f32(NULL, NULL, NULL, NULL, NULL, 1, 90, 3, 256, 18, 1, NULL) == -2  # D > 128
+
+
+def test_rope_validation(lib):
+    assert lib.rope_pi_apply(NULL, NULL, 1, 16, 2, 128, 0.5, 10000.0, NULL) == -1   # neither q nor k
+    p = ctypes.c_void_p(0x1000)
+    assert lib.rope_pi_apply(p, NULL, 1, 16, 2, 100, 0.5, 10000.0, NULL) == -1      # D % 16 != 0
+    assert lib.rope_pi_apply(p, NULL, 1, 16, 2, 128, 0.5, -1.0, NULL) == -1         # bad base
+
+
+def test_workspace_checked_before_launch(lib):
+    p = ctypes.c_void_p(0x10000)
+    rc = lib.s2attn_bwd(p, p, p, p, p, p, p, p, p, 1, 1024, 2, 128, 512, 0, p, 16, NULL)
+    assert rc == -3
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    import shifted_sparse_attention_s2attn_b200 as s2
+    monkeypatch.setattr(s2, "_lib", None)
+    monkeypatch.setattr(s2, "library_path", "/nonexistent/libs2attn.so")
+    with pytest.raises(RuntimeError):
+        s2.capi()
