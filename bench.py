@@ -1,0 +1,392 @@
+#!/usr/bin/env python3
+"""Throughput of the S^2-Attn hot path on B200: useful causal-within-group TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of the synthetic
+LLaMA2-7B layer at N=32768 (B=1, H=32 with 16 shifted heads, D=128, G=8192):
+rope_pi_apply(q, k) -> s2attn_fwd -> s2attn_bwd (preprocess, main, dQ convert).
+Useful FLOPs per step = 3.5 * 4 * D * (causal in-group pairs) (forward 4*D per pair,
+backward 2.5x the forward).  Inputs are resident in HBM and larger than L2.
+
+Multi-GPU (torchrun, one process per GPU): the path does not shard across GPUs
+here, so every rank runs an independent replica of the workload; value counts the
+work of all ranks over the slowest rank's time ("scaling": "weak").
+
+--impl reference times the fp64 CPU oracle (the method's plain definition) on a
+bounded sample of the same workload, on this machine's host cores, rank 0 only.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from shifted_sparse_attention_s2attn_b200.synthetic import WORKLOADS, make_tensor  # noqa: E402
+
+METRIC = "S²-Attn fwd+bwd useful TFLOP/s at LLaMA2-7B shape N=32k (% of bf16 peak)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LAUNCHES_PER_STEP = 5  # rope, fwd, bwd preprocess, bwd main, dQ convert
+
+
+def useful_pairs(w):
+    return w.B * w.H * (w.N // w.G) * w.G * (w.G + 1) // 2
+
+
+def step_flops(w):
+    return 3.5 * 4 * w.D * useful_pairs(w)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------------
+# clocks sampled during the timed region
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_indices):
+        self.gpus = set(gpu_indices)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                idx = int(parts[0])
+            except ValueError:
+                continue
+            if idx not in self.gpus:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                pass
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------
+# the oracle on a bounded sample (CPU baseline and the reference arm)
+def oracle_sample_flops(w, R):
+    """Useful FLOPs of the oracle sample: the last R query rows and the last R key rows of
+    one group, i.e. forward + dQ for every pair whose query is among the R rows
+    (10*D FLOPs per pair) and dK + dV for the pairs inside the R x R triangle (4*D)."""
+    G, D = w.G, w.D
+    q_pairs = sum(range(G - R + 1, G + 1))
+    return 10 * D * q_pairs + 4 * D * R * (R + 1) // 2
+
+
+def run_oracle_sample(w, inputs, R, unit):
+    import oracle
+    b, h, j = unit
+    rows = list(range(w.G - R, w.G))
+    t0 = time.perf_counter()
+    oracle.s2attn_unit(inputs["q"], inputs["k"], inputs["v"], w.G, w.shift_heads, b, h, j, qrows=rows, krows=rows,
+                       dout=inputs["dout"])
+    return time.perf_counter() - t0
+
+
+def oracle_inputs(w):
+    import oracle
+    inp = {n: make_tensor(w, n) for n in ("q", "k", "v", "dout")}
+    inp["q"] = oracle.rope_pi_bf16(inp["q"], w.pos_scale, w.base)
+    inp["k"] = oracle.rope_pi_bf16(inp["k"], w.pos_scale, w.base)
+    return inp
+
+
+def cpu_baseline(w, min_seconds=10.0, max_units=16):
+    """Whole groups (fwd+bwd, every row) of the shifted heads' wrap-around group, until >= min_seconds."""
+    inp = oracle_inputs(w)
+    units = [(0, h, w.groups - 1) for h in range(w.H - 1, -1, -1)]
+    elapsed, flops, n = 0.0, 0.0, 0
+    while n < max_units and (elapsed < min_seconds or n == 0):
+        elapsed += run_oracle_sample(w, inp, w.G, units[n % len(units)])
+        flops += oracle_sample_flops(w, w.G)
+        n += 1
+    return {"value": flops / elapsed / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{n} whole group(s) (G={w.G}, all rows, fwd+bwd) of the {w.name} workload, heads from "
+                      f"H-1 down, last group; fp64 C oracle with OpenMP; {elapsed:.1f} s"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = oracle_inputs(w)
+    unit = (0, w.H - 1, w.groups - 1)
+    # size the per-step sample so that warmup + steps take about two minutes
+    R = 256
+    t = run_oracle_sample(w, inp, R, unit)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    while R < w.G and t < budget / 3:
+        R = min(w.G, R * 2)
+        t = run_oracle_sample(w, inp, R, unit)
+    for _ in range(args.warmup):
+        run_oracle_sample(w, inp, R, unit)
+    total = 0.0
+    for _ in range(args.steps):
+        total += run_oracle_sample(w, inp, R, unit)
+    value = oracle_sample_flops(w, R) * args.steps / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"per step: the last {R} query rows and {R} key rows (fwd+bwd) of group "
+                                   f"{unit[2]} of head {unit[1]} (shifted, wraps around the sequence end)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D, "G": w.G, "shift_heads": w.shift_heads,
+            "rope_pos_scale": w.pos_scale, "step": "rope_pi_apply + s2attn_fwd + s2attn_bwd",
+            "l2": "inputs larger than L2 (q,k,v,dO = %.2f GB)" % (4 * w.B * w.N * w.H * w.D * 2 / 1e9),
+            "parallelism": "replicas"}
+
+
+def traffic_record(kernel_file, kernel):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        recs = json.load(f)
+    src = os.path.join(ROOT, "shifted_sparse_attention_s2attn_b200", "csrc", kernel_file)
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    rec = recs.get(kernel)
+    if not rec or rec.get("source_sha256") != sha:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------------
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import shifted_sparse_attention_s2attn_b200 as s2
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+
+    B, N, H, D, G, SH = w.B, w.N, w.H, w.D, w.G, w.shift_heads
+
+    def to_dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    host = {n: make_tensor(w, n) for n in ("q", "k", "v", "dout")}
+    q, k, v, do = (to_dev(host[n]) for n in ("q", "k", "v", "dout"))
+    o = torch.empty_like(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ws_bytes = s2.s2attn_bwd_workspace_bytes(B, N, H, D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    dq_acc = ws[: B * N * H * D * 4].view(torch.float32)
+    delta_off = ((B * N * H * D * 4 + 255) // 256) * 256
+    delta = ws[delta_off: delta_off + B * H * N * 4].view(torch.float32)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        s2.rope_pi_apply(q, k, w.pos_scale, w.base, stream)
+        if ev is not None:
+            ev[0].record(stream)
+        s2.s2attn_fwd(q, k, v, o, lse, G, SH, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        s2.s2attn_bwd_preprocess(o, do, delta, dq_acc, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        s2.s2attn_bwd_main(q, k, v, do, lse, delta, dq_acc, dk, dv, G, SH, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        s2.s2attn_bwd_dq_convert(dq_acc, dq, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    s2.clear_device_error()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(range(world)) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    barrier()
+    ms = start.elapsed_time(end)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    rc, detail = s2.get_device_error()
+    if rc != 0:
+        raise SystemExit(f"device error word set during the timed region: {detail:#x}")
+
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # ---- end to end: host buffers in, results out, through the same public calls ----
+    e2e_steps = max(3, min(args.steps, 10))
+    pinned = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in host}
+    outs = {n: torch.empty((B, N, H, D), dtype=torch.bfloat16).pin_memory() for n in ("o", "dq", "dk", "dv")}
+    dev_in = {"q": q, "k": k, "v": v, "dout": do}
+    dev_out = {"o": o, "dq": dq, "dk": dk, "dv": dv}
+    h2d = sum(x.numel() * x.element_size() for x in pinned.values())
+    d2h = sum(x.numel() * x.element_size() for x in outs.values())
+
+    def e2e_step():
+        for n in pinned:
+            dev_in[n].copy_(pinned[n], non_blocking=True)
+        step()
+        for n in outs:
+            outs[n].copy_(dev_out[n], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    flops = step_flops(w)
+    value = world * flops * args.steps / (ms_max / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    fwd_flops, bwd_flops = 4 * D * useful_pairs(w), 10 * D * useful_pairs(w)
+    bwd_avg = statistics.mean(bwd_ms) / 1e3
+    fwd_avg = statistics.mean(fwd_ms) / 1e3
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    achieved = bwd_flops / bwd_avg / 1e12
+    traffic = traffic_record("s2attn_bwd_sm100.cu", "s2attn_bwd_kernel")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w),
+        "pct_of_peak": 100.0 * value / world / peak_sus,
+        "peak_used": {"bf16_tflops_sustained": peak_sus, "source": peak_src},
+        "fwd": {"ms": 1e3 * fwd_avg, "tflops": fwd_flops / fwd_avg / 1e12},
+        "bwd_main": {"ms": 1e3 * bwd_avg, "tflops": achieved},
+        "roofline": {"kernel": "s2attn_bwd_kernel", "bound": "tensor", "achieved": achieved, "peak": peak_sus,
+                     "unit": "TFLOP/s", "frac": achieved / peak_sus, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)"},
+        "roofline_fwd": {"kernel": "s2attn_fwd_kernel", "bound": "tensor",
+                         "achieved": fwd_flops / fwd_avg / 1e12, "peak": peak_sus, "unit": "TFLOP/s",
+                         "frac": fwd_flops / fwd_avg / 1e12 / peak_sus,
+                         "traffic": traffic_record("s2attn_fwd_sm100.cu", "s2attn_fwd_kernel")},
+        "e2e": {"value": world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama2_7b_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if w.dtype != "bf16":
+        raise SystemExit("the bench times the bf16 tensor-core path")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

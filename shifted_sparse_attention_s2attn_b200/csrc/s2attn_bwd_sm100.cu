@@ -16,7 +16,9 @@
 //   dV += P^T dO  (P^T from TMEM), dK += dS^T Q   (M=128 keys, N=128 dims)
 //   dQ^T = K^T dS^T                               (M=128 dims, N=64 queries)
 // dQ^T leaves TMEM through shared memory and is added into an fp32 accumulator in
-// global memory by one TMA reduce-add per step.  Items run heaviest first (kt = 0).
+// global memory by one TMA reduce-add per step.  Each CTA runs two key tiles of one
+// group, kt and n_kt-1-kt, so every CTA walks the same number of query steps, and
+// consecutive CTAs share a group: its Q, dO and dQ accumulator rows stay in L2.
 //
 // Warp roles (320 threads):
 //   warps 0-3  P / dS: thread = key row (TMEM lanes); writes P^T into TMEM and dS^T
@@ -50,8 +52,8 @@ constexpr uint32_t OFF_DQ = OFF_DS + 2 * DS_BYTES;
 constexpr uint32_t DQ_BYTES = BQ * HD * 4;  // fp32 staging tile
 constexpr uint32_t OFF_BAR = OFF_DQ + DQ_BYTES;
 // kv_full, q_full[2], q_empty[2], s_full, dp_full, p_ready, ds_ready, ds_free[2], dq_full, dq_free,
-// mma_done, drain
-constexpr int NBARS = 15;
+// mma_done, drain, kv_empty, dkv_empty
+constexpr int NBARS = 17;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
 constexpr int NTHREADS = 320;
@@ -102,30 +104,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* dq_free = bars + 12;
   uint64_t* mma_done = bars + 13;
   uint64_t* drain = bars + 14;
+  uint64_t* kv_empty = bars + 15;
+  uint64_t* dkv_empty = bars + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // ---- work item -------------------------------------------------------------
-  const int per_kt = p.B * p.H * p.n_groups;
-  const int kt = (int)(blockIdx.x / per_kt);
-  int rest = (int)(blockIdx.x % per_kt);
-  const int j = rest % p.n_groups;
-  rest /= p.n_groups;
-  const int h = rest % p.H;
-  const int b = rest / p.H;
-  const int nsteps = p.G / BQ - 2 * kt;   // query steps of 64 rows: local rows 128*kt .. G-1
+  // ---- work items: one group (b, h, j); key tiles kt0 (heavy) and n_kt-1-kt0 (light) ----
+  const int n_fold = (p.n_kt + 1) / 2;
+  const int unit = (int)(blockIdx.x / n_fold);
+  const int fi = (int)(blockIdx.x % n_fold);
+  const int j = unit % p.n_groups;
+  const int h = (unit / p.n_groups) % p.H;
+  const int b = unit / (p.n_groups * p.H);
+  int kts[2];
+  int n_items = 0;
+  kts[n_items++] = fi;
+  if (fi != p.n_kt - 1 - fi) kts[n_items++] = p.n_kt - 1 - fi;
   const int shift = (h >= p.H - p.shift_heads) ? p.G / 2 : 0;
   const int group_row0 = j * p.G;
   auto token_of = [&](int local_row) {  // original token of a local (rolled) row; tiles never wrap
     int t = group_row0 + local_row + shift;
     return t >= p.N ? t - p.N : t;
   };
-  const int key_tok0 = token_of(kt * BK);
+  auto steps_of = [&](int kt) { return p.G / BQ - 2 * kt; };  // query steps of 64 rows: rows 128*kt .. G-1
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
     for (int s = 0; s < QSTAGES; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
@@ -138,6 +145,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 4);
     mbar_init(mma_done, 1);
+    mbar_init(dkv_empty, 4);
     mbar_init(drain, 1);
     *abort_flag = (*(volatile int*)p.err != 0) ? 1 : 0;
     fence_mbar_init();
@@ -160,36 +168,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tdo);
     bool ok = true;
     const int row_base = b * p.N;
-    mbar_arrive_expect_tx(kv_full, 2 * KTILE);
-    for (int x = 0; x < 2; ++x) {
-      tma_load_3d(smem + OFF_K + x * KBOX, &tk, x * 64, h, row_base + key_tok0, kv_full);
-      tma_load_3d(smem + OFF_V + x * KBOX, &tv, x * 64, h, row_base + key_tok0, kv_full);
-    }
     const size_t stat_base = ((size_t)b * p.H + h) * p.N;
-    int armed = 0;
-    for (int it = 0; it < nsteps; ++it) {
-      const int st = it % QSTAGES;
-      const uint32_t ph = (it / QSTAGES) & 1;
-      ok = wait_bounded(&q_empty[st], ph ^ 1, abort_flag, p.err);
-      if (!ok) break;
-      uint8_t* stage = smem + OFF_STAGE + st * STAGE_BYTES;
-      const int tok = token_of((2 * kt + it) * BQ);
-      mbar_arrive_expect_tx(&q_full[st], 2 * QTILE + 512);
-      for (int x = 0; x < 2; ++x) {
-        tma_load_3d(stage + ST_Q + x * QBOX, &tq, x * 64, h, row_base + tok, &q_full[st]);
-        tma_load_3d(stage + ST_DO + x * QBOX, &tdo, x * 64, h, row_base + tok, &q_full[st]);
+    int kv_loads = 0, q_armed = 0;
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int kt = kts[it];
+      if (it > 0) {
+        ok = wait_bounded(kv_empty, (it - 1) & 1, abort_flag, p.err);
+        if (!ok) break;
       }
-      bulk_load(stage + ST_LSE, p.lse + stat_base + tok, 256, &q_full[st]);
-      bulk_load(stage + ST_DELTA, p.delta + stat_base + tok, 256, &q_full[st]);
-      armed = it + 1;
+      const int key_tok0 = token_of(kt * BK);
+      mbar_arrive_expect_tx(kv_full, 2 * KTILE);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_3d(smem + OFF_K + x * KBOX, &tk, x * 64, h, row_base + key_tok0, kv_full);
+        tma_load_3d(smem + OFF_V + x * KBOX, &tv, x * 64, h, row_base + key_tok0, kv_full);
+      }
+      ++kv_loads;
+      const int nsteps = steps_of(kt);
+      for (int s = 0; s < nsteps; ++s) {
+        const int g = q_armed;
+        const int st = g % QSTAGES;
+        ok = wait_bounded(&q_empty[st], ((g / QSTAGES) & 1) ^ 1, abort_flag, p.err);
+        if (!ok) break;
+        uint8_t* stage = smem + OFF_STAGE + st * STAGE_BYTES;
+        const int tok = token_of((2 * kt + s) * BQ);
+        mbar_arrive_expect_tx(&q_full[st], 2 * QTILE + 512);
+        for (int x = 0; x < 2; ++x) {
+          tma_load_3d(stage + ST_Q + x * QBOX, &tq, x * 64, h, row_base + tok, &q_full[st]);
+          tma_load_3d(stage + ST_DO + x * QBOX, &tdo, x * 64, h, row_base + tok, &q_full[st]);
+        }
+        bulk_load(stage + ST_LSE, p.lse + stat_base + tok, 256, &q_full[st]);
+        bulk_load(stage + ST_DELTA, p.delta + stat_base + tok, 256, &q_full[st]);
+        q_armed = g + 1;
+      }
     }
     if (!ok) {
       report_error(p.err, (K_BWD << 8) | SITE_LOAD);
       *abort_flag = 1;
     }
-    bool dok = wait_drain(kv_full, 0);
-    for (int it = (armed > QSTAGES ? armed - QSTAGES : 0); it < armed; ++it)
-      dok &= wait_drain(&q_full[it % QSTAGES], (it / QSTAGES) & 1);
+    bool dok = kv_loads == 0 || wait_drain(kv_full, (kv_loads - 1) & 1);
+    for (int g = (q_armed > QSTAGES ? q_armed - QSTAGES : 0); g < q_armed; ++g)
+      dok &= wait_drain(&q_full[g % QSTAGES], (g / QSTAGES) & 1);
     if (!dok) report_error(p.err, (K_BWD << 8) | SITE_DRAIN);
   } else if (!skip && warp == WARP_MMA && lane == 0) {
     // ---------------- MMA issuer ----------------
@@ -198,66 +216,74 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t id_dq = idesc_bf16_f32(HD, BQ, true, true);     // dQ^T = K^T dS^T
     const uint32_t sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
     const uint32_t sstage = smem_u32(smem + OFF_STAGE), sds = smem_u32(smem + OFF_DS);
-    bool ok = wait_bounded(kv_full, 0, abort_flag, p.err);
-    if (ok) ok = wait_bounded(&q_full[0], 0, abort_flag, p.err);
-    if (ok) {
+    bool ok = true;
+    int g0 = 0;  // global index of the current item's first query step
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int nsteps = steps_of(kts[it]);
+      ok = wait_bounded(kv_full, it & 1, abort_flag, p.err);
+      if (ok) ok = wait_bounded(&q_full[g0 % QSTAGES], (g0 / QSTAGES) & 1, abort_flag, p.err);
+      if (!ok) break;
       tc_fence_after();
-      issue_kq(tmem + TM_S, sk, sstage + ST_Q, id_kq);
+      issue_kq(tmem + TM_S, sk, sstage + (g0 % QSTAGES) * STAGE_BYTES + ST_Q, id_kq);
       mma_commit(s_full);
-      issue_kq(tmem + TM_DP, sv, sstage + ST_DO, id_kq);
+      issue_kq(tmem + TM_DP, sv, sstage + (g0 % QSTAGES) * STAGE_BYTES + ST_DO, id_kq);
       mma_commit(dp_full);
-    }
-    for (int it = 0; it < nsteps && ok; ++it) {
-      const int st = it % QSTAGES;
-      const uint32_t sq = sstage + st * STAGE_BYTES + ST_Q, sdo = sstage + st * STAGE_BYTES + ST_DO;
-      const uint32_t sdst = sds + st * DS_BYTES;
-      // dV += P^T dO
-      ok = wait_bounded(p_ready, it & 1, abort_flag, p.err);
-      if (!ok) break;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < BQ / 16; ++kk)
-        mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8, sdesc_sw128(sdo + kk * 2048, QBOX, 1024), id_dkv,
-               (it > 0 || kk > 0) ? 1u : 0u);
-      // next S^T (its columns held P^T, which the dV MMAs above read first: in-order issue)
-      if (it + 1 < nsteps) {
-        const int st1 = (it + 1) % QSTAGES;
-        ok = wait_bounded(&q_full[st1], ((it + 1) / QSTAGES) & 1, abort_flag, p.err);
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int g = g0 + s;
+        const int st = g % QSTAGES;
+        const uint32_t sq = sstage + st * STAGE_BYTES + ST_Q, sdo = sstage + st * STAGE_BYTES + ST_DO;
+        const uint32_t sdst = sds + st * DS_BYTES;
+        // dV += P^T dO
+        ok = wait_bounded(p_ready, g & 1, abort_flag, p.err);
+        if (ok && s == 0 && it > 0) ok = wait_bounded(dkv_empty, (it - 1) & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
-        issue_kq(tmem + TM_S, sk, sstage + st1 * STAGE_BYTES + ST_Q, id_kq);
-        mma_commit(s_full);
-      }
-      // dK += dS^T Q ; dQ^T = K^T dS^T
-      ok = wait_bounded(ds_ready, it & 1, abort_flag, p.err);
-      if (!ok) break;
-      tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < BQ / 16; ++kk)
-        mma_ss(tmem + TM_DK, sdesc_sw128(sdst + kk * 32, 16, 1024), sdesc_sw128(sq + kk * 2048, QBOX, 1024), id_dkv,
-               (it > 0 || kk > 0) ? 1u : 0u);
-      if (it > 0) {
-        ok = wait_bounded(dq_free, (it - 1) & 1, abort_flag, p.err);
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8, sdesc_sw128(sdo + kk * 2048, QBOX, 1024), id_dkv,
+                 (s > 0 || kk > 0) ? 1u : 0u);
+        // next S^T (its columns held P^T, which the dV MMAs above read first: in-order issue)
+        if (s + 1 < nsteps) {
+          const int st1 = (g + 1) % QSTAGES;
+          ok = wait_bounded(&q_full[st1], ((g + 1) / QSTAGES) & 1, abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+          issue_kq(tmem + TM_S, sk, sstage + st1 * STAGE_BYTES + ST_Q, id_kq);
+          mma_commit(s_full);
+        }
+        // dK += dS^T Q ; dQ^T = K^T dS^T
+        ok = wait_bounded(ds_ready, g & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
-      }
 #pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk)
-        mma_ss(tmem + TM_DQ, sdesc_sw128(sk + kk * 2048, KBOX, 1024), sdesc_sw128(sdst + kk * 2048, QBOX, 1024),
-               id_dq, kk > 0 ? 1u : 0u);
-      mma_commit(dq_full);
-      mma_commit(&ds_free[st]);
-      mma_commit(&q_empty[st]);
-      // next dP^T (the P/dS warps finished reading dP^T before signalling ds_ready)
-      if (it + 1 < nsteps) {
-        const int st1 = (it + 1) % QSTAGES;
-        issue_kq(tmem + TM_DP, sv, sstage + st1 * STAGE_BYTES + ST_DO, id_kq);
-        mma_commit(dp_full);
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          mma_ss(tmem + TM_DK, sdesc_sw128(sdst + kk * 32, 16, 1024), sdesc_sw128(sq + kk * 2048, QBOX, 1024),
+                 id_dkv, (s > 0 || kk > 0) ? 1u : 0u);
+        if (g > 0) {
+          ok = wait_bounded(dq_free, (g - 1) & 1, abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_ss(tmem + TM_DQ, sdesc_sw128(sk + kk * 2048, KBOX, 1024), sdesc_sw128(sdst + kk * 2048, QBOX, 1024),
+                 id_dq, kk > 0 ? 1u : 0u);
+        mma_commit(dq_full);
+        mma_commit(&ds_free[st]);
+        mma_commit(&q_empty[st]);
+        // next dP^T (the P/dS warps finished reading dP^T before signalling ds_ready)
+        if (s + 1 < nsteps) {
+          const int st1 = (g + 1) % QSTAGES;
+          issue_kq(tmem + TM_DP, sv, sstage + st1 * STAGE_BYTES + ST_DO, id_kq);
+          mma_commit(dp_full);
+        }
       }
+      if (!ok) break;
+      mma_commit(mma_done);  // dK, dV of this item complete
+      mma_commit(kv_empty);  // K, V no longer read
+      g0 += nsteps;
     }
-    if (ok) {
-      mma_commit(mma_done);
-    } else {
+    if (!ok) {
       report_error(p.err, (K_BWD << 8) | SITE_MMA);
       *abort_flag = 1;
     }
@@ -266,76 +292,77 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (!skip && warp < 4) {
     // ---------------- P / dS warps: thread = key row ----------------
     const int kr = warp * 32 + lane;
-    const int key_local = kt * BK + kr;
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     const float sl2 = p.sl2;
     bool ok = true;
-    for (int it = 0; it < nsteps && ok; ++it) {
-      const int st = it % QSTAGES;
-      const int q_local0 = (2 * kt + it) * BQ;
-      const float* lse_s = reinterpret_cast<const float*>(smem + OFF_STAGE + st * STAGE_BYTES + ST_LSE);
-      const float* delta_s = reinterpret_cast<const float*>(smem + OFF_STAGE + st * STAGE_BYTES + ST_DELTA);
-      ok = wait_bounded(&q_full[st], (it / QSTAGES) & 1, abort_flag, p.err);
-      if (ok) ok = wait_bounded(s_full, it & 1, abort_flag, p.err);
-      if (!ok) break;
-      tc_fence_after();
-      float pr[64];
-      {
-        uint32_t sr[64];
-        tmem_ld_x64(lane_addr + TM_S, sr);
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float e = ex2_approx(__uint_as_float(sr[c]) * sl2 - lse_s[c] * LOG2E);
-          pr[c] = (key_local > q_local0 + c) ? 0.0f : e;   // causal: key after query -> masked
-        }
-      }
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-        tmem_st_x32(lane_addr + TM_S, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_ready);
-
-      ok = wait_bounded(dp_full, it & 1, abort_flag, p.err);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t pk[32];
-      {
-        uint32_t dr[64];
-        tmem_ld_x64(lane_addr + TM_DP, dr);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float d0 = pr[2 * c] * (__uint_as_float(dr[2 * c]) - delta_s[2 * c]);
-          const float d1 = pr[2 * c + 1] * (__uint_as_float(dr[2 * c + 1]) - delta_s[2 * c + 1]);
-          pk[c] = pack_bf16x2(d0, d1);
-        }
-      }
-      tc_fence_before();
-      if (it >= QSTAGES) {
-        ok = wait_bounded(&ds_free[st], ((it - QSTAGES) / QSTAGES) & 1, abort_flag, p.err);
+    int g = 0;
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int kt = kts[it];
+      const int nsteps = steps_of(kt);
+      const int key_local = kt * BK + kr;
+      for (int s = 0; s < nsteps; ++s, ++g) {
+        const int st = g % QSTAGES;
+        const int q_local0 = (2 * kt + s) * BQ;
+        const float* lse_s = reinterpret_cast<const float*>(smem + OFF_STAGE + st * STAGE_BYTES + ST_LSE);
+        const float* delta_s = reinterpret_cast<const float*>(smem + OFF_STAGE + st * STAGE_BYTES + ST_DELTA);
+        ok = wait_bounded(&q_full[st], (g / QSTAGES) & 1, abort_flag, p.err);
+        if (ok) ok = wait_bounded(s_full, g & 1, abort_flag, p.err);
         if (!ok) break;
-      }
-      // dS^T row kr: 64 bf16 = 8 chunks of 16 B, chunk c stored at chunk slot c ^ (kr % 8)
-      uint8_t* dsrow = smem + OFF_DS + st * DS_BYTES + kr * 128;
+        tc_fence_after();
+        float pr[64];
+        {
+          uint32_t sr[64];
+          tmem_ld_x64(lane_addr + TM_S, sr);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(dsrow + ((c ^ (kr & 7)) * 16)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ds_ready);
-    }
-    if (ok) ok = wait_bounded(mma_done, 0, abort_flag, p.err);
-    if (!ok) {
-      report_error(p.err, (K_BWD << 8) | SITE_PDS);
-      *abort_flag = 1;
-    } else {
+          for (int c = 0; c < 64; ++c) {
+            const float e = ex2_approx(__uint_as_float(sr[c]) * sl2 - lse_s[c] * LOG2E);
+            pr[c] = (key_local > q_local0 + c) ? 0.0f : e;  // causal: key after query -> masked
+          }
+        }
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+          tmem_st_x32(lane_addr + TM_S, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_ready);
+
+        ok = wait_bounded(dp_full, g & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t pk[32];
+        {
+          uint32_t dr[64];
+          tmem_ld_x64(lane_addr + TM_DP, dr);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float d0 = pr[2 * c] * (__uint_as_float(dr[2 * c]) - delta_s[2 * c]);
+            const float d1 = pr[2 * c + 1] * (__uint_as_float(dr[2 * c + 1]) - delta_s[2 * c + 1]);
+            pk[c] = pack_bf16x2(d0, d1);
+          }
+        }
+        tc_fence_before();
+        if (g >= QSTAGES) {
+          ok = wait_bounded(&ds_free[st], ((g - QSTAGES) / QSTAGES) & 1, abort_flag, p.err);
+          if (!ok) break;
+        }
+        // dS^T row kr: 64 bf16 = 8 chunks of 16 B, chunk c stored at chunk slot c ^ (kr % 8)
+        uint8_t* dsrow = smem + OFF_DS + st * DS_BYTES + kr * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(dsrow + ((c ^ (kr & 7)) * 16)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_ready);
+      }
+      if (ok) ok = wait_bounded(mma_done, it & 1, abort_flag, p.err);
+      if (!ok) break;
       tc_fence_after();
-      const int tok = key_tok0 + kr;
+      const int tok = token_of(kt * BK) + kr;
       __nv_bfloat16* dkrow = p.dk + ((size_t)(b * p.N + tok) * p.H + h) * HD;
       __nv_bfloat16* dvrow = p.dv + ((size_t)(b * p.N + tok) * p.H + h) * HD;
 #pragma unroll
@@ -355,6 +382,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dkv_empty);
+    }
+    if (!ok) {
+      report_error(p.err, (K_BWD << 8) | SITE_PDS);
+      *abort_flag = 1;
     }
   } else if (!skip && warp >= 4 && warp < 8) {
     // ---------------- dQ drain: thread = head dim ----------------
@@ -363,24 +397,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)((warp - 4) * 32) << 16);
     float* stage = reinterpret_cast<float*>(smem + OFF_DQ);
     bool ok = true;
-    for (int it = 0; it < nsteps && ok; ++it) {
-      ok = wait_bounded(dq_full, it & 1, abort_flag, p.err);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t r[64];
-      tmem_ld_x64(lane_addr + TM_DQ, r);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
-      if (leader && it > 0) bulk_wait_group_read0();  // previous reduce finished reading the staging tile
-      named_bar_sync(1, 128);
+    int g = 0;
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int kt = kts[it];
+      const int nsteps = steps_of(kt);
+      for (int s = 0; s < nsteps; ++s, ++g) {
+        ok = wait_bounded(dq_full, g & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t r[64];
+        tmem_ld_x64(lane_addr + TM_DQ, r);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free);
+        if (leader && g > 0) bulk_wait_group_read0();  // previous reduce finished reading the staging tile
+        named_bar_sync(1, 128);
 #pragma unroll
-      for (int c = 0; c < BQ; ++c) stage[c * HD + d] = __uint_as_float(r[c]);
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (leader) {
-        tma_reduce_add_3d(&tdq, stage, 0, h, b * p.N + token_of((2 * kt + it) * BQ));
-        bulk_commit_group();
+        for (int c = 0; c < BQ; ++c) stage[c * HD + d] = __uint_as_float(r[c]);
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader) {
+          tma_reduce_add_3d(&tdq, stage, 0, h, b * p.N + token_of((2 * kt + s) * BQ));
+          bulk_commit_group();
+        }
       }
     }
     if (leader) bulk_wait_group0();
@@ -418,7 +457,7 @@ cudaError_t launch_bwd_sm100(const CUtensorMap& tq64, const CUtensorMap& tk, con
   p.scale = (float)(1.0 / sqrt((double)s.D));
   p.sl2 = (float)(1.4426950408889634 / sqrt((double)s.D));
   p.err = err;
-  const long long grid = (long long)p.n_kt * s.B * s.H * p.n_groups;
+  const long long grid = (long long)((p.n_kt + 1) / 2) * s.B * s.H * p.n_groups;
   if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(bwd::s2attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bwd::SMEM_BYTES);

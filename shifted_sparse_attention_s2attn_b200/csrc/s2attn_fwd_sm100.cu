@@ -12,10 +12,12 @@
 // and each output row is stored straight back to its original token: no rolled copy
 // of Q/K/V/O ever exists.
 //
-// CTA work item: (batch b, head h, group j, pair m) -> the two query tiles 2m and
-// 2m+1 of the group (128 rows each), which share every K/V tile they load.  Only the
-// causal lower triangle is visited: query tile qt needs key tiles 0..qt, and only
-// tile qt (the diagonal) is masked.  Items are ordered heaviest first.
+// Work item: (batch b, head h, group j, pair m) -> the two query tiles 2m and 2m+1 of
+// the group (128 rows each), which share every K/V tile they load.  Only the causal
+// lower triangle is visited: query tile qt needs key tiles 0..qt, and only tile qt
+// (the diagonal) is masked.  Each CTA runs two items of one group, pair m and pair
+// n_pairs-1-m, so every CTA does the same number of K/V tiles; consecutive CTAs
+// share a group, which keeps that group's K/V resident in L2.
 //
 // Warp roles (320 threads):
 //   warps 0-3  softmax for query tile 0 (thread = row; TMEM lanes 0..127)
@@ -51,8 +53,9 @@ constexpr uint32_t OFF_Q1 = OFF_Q0 + TILE_BYTES;
 constexpr uint32_t OFF_K = OFF_Q1 + TILE_BYTES;
 constexpr uint32_t OFF_V = OFF_K + STAGES * TILE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE_BYTES;
-// barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_ready[2], o_final[2], drain
-constexpr int NBARS = 16;
+// barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_ready[2], o_final[2], drain,
+// q_empty, o_empty[2]
+constexpr int NBARS = 19;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
 
@@ -103,22 +106,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* p_ready = bars + 11;
   uint64_t* o_final = bars + 13;
   uint64_t* drain = bars + 15;
+  uint64_t* q_empty = bars + 16;
+  uint64_t* o_empty = bars + 17;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // ---- work item -------------------------------------------------------------
-  const int per_m = p.B * p.H * p.n_groups;
-  const int m = p.n_pairs - 1 - (int)(blockIdx.x / per_m);
-  int rest = (int)(blockIdx.x % per_m);
-  const int j = rest % p.n_groups;
-  rest /= p.n_groups;
-  const int h = rest % p.H;
-  const int b = rest / p.H;
-  const int qa = 2 * m, qb = 2 * m + 1;
-  const bool has_b = qb < p.n_qt;
-  const int nkv = (has_b ? qb : qa) + 1;
+  // ---- work items: one group (b, h, j); the heavy tile pair m0 and the light pair m1 ----
+  const int n_fold = (p.n_pairs + 1) / 2;
+  const int unit = (int)(blockIdx.x / n_fold);
+  const int fi = (int)(blockIdx.x % n_fold);
+  const int j = unit % p.n_groups;
+  const int h = (unit / p.n_groups) % p.H;
+  const int b = unit / (p.n_groups * p.H);
+  int ms[2];
+  int n_items = 0;
+  ms[n_items++] = p.n_pairs - 1 - fi;
+  if (fi != p.n_pairs - 1 - fi) ms[n_items++] = fi;
   const int shift = (h >= p.H - p.shift_heads) ? p.G / 2 : 0;
   const int group_row0 = j * p.G;
   // first original token of the 128-row tile `tile` of this group (tiles never wrap)
@@ -129,6 +134,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -139,6 +145,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&p_ready[i], 4);
       mbar_init(&o_final[i], 1);
+      mbar_init(&o_empty[i], 4);
     }
     mbar_init(drain, 1);
     *abort_flag = (*(volatile int*)p.err != 0) ? 1 : 0;  // an earlier CTA failed: skip the work
@@ -161,38 +168,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tv);
     bool ok = true;
     const int row_base = b * p.N;
-    mbar_arrive_expect_tx(q_full, (has_b ? 2u : 1u) * TILE_BYTES);
-    for (int x = 0; x < NBOX; ++x) {
-      tma_load_3d(smem + OFF_Q0 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(qa), q_full);
-      if (has_b) tma_load_3d(smem + OFF_Q1 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(qb), q_full);
-    }
-    int armed = 0;  // K/V tiles issued
-    for (int t = 0; t < nkv && ok; ++t) {
-      const int st = t % STAGES;
-      const uint32_t ph = (t / STAGES) & 1;
-      const int row = row_base + tile_token0(t);
-      ok = wait_bounded(&k_empty[st], ph ^ 1, abort_flag, p.err);
-      if (!ok) break;
-      mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
-      for (int x = 0; x < NBOX; ++x) tma_load_3d(smem + OFF_K + st * TILE_BYTES + x * BOX_BYTES, &tk, x * 64, h, row, &k_full[st]);
-      ok = wait_bounded(&v_empty[st], ph ^ 1, abort_flag, p.err);
-      if (!ok) {
-        armed = -(t + 1);  // K of tile t in flight, V not
-        break;
+    int q_loads = 0, kv = 0, k_armed = 0, v_armed = 0;  // loads issued
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int qa = 2 * ms[it], qb = qa + 1;
+      const bool has_b = qb < p.n_qt;
+      const int nkv = (has_b ? qb : qa) + 1;
+      if (it > 0) {
+        ok = wait_bounded(q_empty, (it - 1) & 1, abort_flag, p.err);
+        if (!ok) break;
       }
-      mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
-      for (int x = 0; x < NBOX; ++x) tma_load_3d(smem + OFF_V + st * TILE_BYTES + x * BOX_BYTES, &tv, x * 64, h, row, &v_full[st]);
-      armed = t + 1;
+      mbar_arrive_expect_tx(q_full, (has_b ? 2u : 1u) * TILE_BYTES);
+      for (int x = 0; x < NBOX; ++x) {
+        tma_load_3d(smem + OFF_Q0 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(qa), q_full);
+        if (has_b) tma_load_3d(smem + OFF_Q1 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(qb), q_full);
+      }
+      ++q_loads;
+      for (int t = 0; t < nkv; ++t, ++kv) {
+        const int st = kv % STAGES;
+        const uint32_t ph = (kv / STAGES) & 1;
+        const int row = row_base + tile_token0(t);
+        ok = wait_bounded(&k_empty[st], ph ^ 1, abort_flag, p.err);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
+        for (int x = 0; x < NBOX; ++x)
+          tma_load_3d(smem + OFF_K + st * TILE_BYTES + x * BOX_BYTES, &tk, x * 64, h, row, &k_full[st]);
+        k_armed = kv + 1;
+        ok = wait_bounded(&v_empty[st], ph ^ 1, abort_flag, p.err);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
+        for (int x = 0; x < NBOX; ++x)
+          tma_load_3d(smem + OFF_V + st * TILE_BYTES + x * BOX_BYTES, &tv, x * 64, h, row, &v_full[st]);
+        v_armed = kv + 1;
+      }
     }
     if (!ok) {
       report_error(p.err, (K_FWD << 8) | SITE_LOAD);
       *abort_flag = 1;
     }
     // Drain: every copy this thread started must land before the CTA can exit.
-    bool dok = wait_drain(q_full, 0);
-    const int nk = armed >= 0 ? armed : -armed, nv = armed >= 0 ? armed : -armed - 1;
-    for (int t = (nk > STAGES ? nk - STAGES : 0); t < nk; ++t) dok &= wait_drain(&k_full[t % STAGES], (t / STAGES) & 1);
-    for (int t = (nv > STAGES ? nv - STAGES : 0); t < nv; ++t) dok &= wait_drain(&v_full[t % STAGES], (t / STAGES) & 1);
+    bool dok = q_loads == 0 || wait_drain(q_full, (q_loads - 1) & 1);
+    for (int t = (k_armed > STAGES ? k_armed - STAGES : 0); t < k_armed; ++t)
+      dok &= wait_drain(&k_full[t % STAGES], (t / STAGES) & 1);
+    for (int t = (v_armed > STAGES ? v_armed - STAGES : 0); t < v_armed; ++t)
+      dok &= wait_drain(&v_full[t % STAGES], (t / STAGES) & 1);
     if (!dok) report_error(p.err, (K_FWD << 8) | SITE_DRAIN);
   } else if (!skip && warp == WARP_MMA && lane == 0) {
     // ---------------- MMA issuer ----------------
@@ -200,34 +218,50 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t id_pv = idesc_bf16_f32(BM, HD, false, true);
     const uint32_t sq[2] = {smem_u32(smem + OFF_Q0), smem_u32(smem + OFF_Q1)};
     const uint32_t sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
-    const int qts[2] = {qa, qb};
     uint32_t p_phase[2] = {0, 0};
-    bool ok = wait_bounded(q_full, 0, abort_flag, p.err);
-    for (int t = 0; t <= nkv && ok; ++t) {
-      const bool has_prev = t > 0, has_cur = t < nkv;
-      if (has_cur) ok = wait_bounded(&k_full[t % STAGES], (t / STAGES) & 1, abort_flag, p.err);
-      if (ok && has_prev) ok = wait_bounded(&v_full[(t - 1) % STAGES], ((t - 1) / STAGES) & 1, abort_flag, p.err);
-      if (!ok) break;
-      tc_fence_after();
-      for (int i = 0; i < 2 && ok; ++i) {
-        if (i == 1 && !has_b) break;
-        const int qt = qts[i];
-        if (has_prev && t - 1 <= qt) {
-          ok = wait_bounded(&p_ready[i], p_phase[i], abort_flag, p.err);
-          p_phase[i] ^= 1;
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(tmem + tm_o(i), tmem + tm_s(i), sv + ((t - 1) % STAGES) * TILE_BYTES, id_pv, t - 1 == 0);
-          if (t - 1 == qt) mma_commit(&o_final[i]);
+    int o_items[2] = {0, 0};  // items whose O_i has been produced
+    int kv0 = 0;              // K/V ring position of tile 0 of the current item
+    bool ok = true;
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int qa = 2 * ms[it], qb = qa + 1;
+      const bool has_b = qb < p.n_qt;
+      const int nkv = (has_b ? qb : qa) + 1;
+      const int qts[2] = {qa, qb};
+      ok = wait_bounded(q_full, it & 1, abort_flag, p.err);
+      for (int t = 0; t <= nkv && ok; ++t) {
+        const bool has_prev = t > 0, has_cur = t < nkv;
+        const int g = kv0 + t;  // ring position of K/V tile t
+        if (has_cur) ok = wait_bounded(&k_full[g % STAGES], (g / STAGES) & 1, abort_flag, p.err);
+        if (ok && has_prev) ok = wait_bounded(&v_full[(g - 1) % STAGES], ((g - 1) / STAGES) & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (i == 1 && !has_b) break;
+          const int qt = qts[i];
+          if (has_prev && t - 1 <= qt) {
+            ok = wait_bounded(&p_ready[i], p_phase[i], abort_flag, p.err);
+            p_phase[i] ^= 1;
+            if (ok && t == 1 && o_items[i] > 0)  // O_i of the previous item read out by its epilogue
+              ok = wait_bounded(&o_empty[i], (o_items[i] - 1) & 1, abort_flag, p.err);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(tmem + tm_o(i), tmem + tm_s(i), sv + ((g - 1) % STAGES) * TILE_BYTES, id_pv, t == 1);
+            if (t - 1 == qt) {
+              mma_commit(&o_final[i]);
+              ++o_items[i];
+            }
+          }
+          if (has_cur && t <= qt) {
+            issue_s(tmem + tm_s(i), sq[i], sk + (g % STAGES) * TILE_BYTES, id_s);
+            mma_commit(&s_full[i]);
+          }
         }
-        if (has_cur && t <= qt) {
-          issue_s(tmem + tm_s(i), sq[i], sk + (t % STAGES) * TILE_BYTES, id_s);
-          mma_commit(&s_full[i]);
-        }
+        if (!ok) break;
+        if (has_prev) mma_commit(&v_empty[(g - 1) % STAGES]);
+        if (has_cur) mma_commit(&k_empty[g % STAGES]);
+        if (t == nkv - 1) mma_commit(q_empty);  // the item's last S MMAs read Q for the last time
       }
-      if (!ok) break;
-      if (has_prev) mma_commit(&v_empty[(t - 1) % STAGES]);
-      if (has_cur) mma_commit(&k_empty[t % STAGES]);
+      kv0 += nkv;
     }
     if (!ok) {
       report_error(p.err, (K_FWD << 8) | SITE_MMA);
@@ -239,93 +273,111 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (!skip && warp < 8) {
     // ---------------- softmax warpgroups ----------------
     const int i = warp / 4;
-    if (i == 0 || has_b) {
+    const int row = (warp % 4) * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
+    const uint32_t t_s = lane_addr + tm_s(i), t_o = lane_addr + tm_o(i);
+    const float sl2 = p.sl2;
+    uint32_t s_phase = 0;
+    int o_items = 0;
+    bool ok = true;
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int qa = 2 * ms[it], qb = qa + 1;
+      const bool has_b = qb < p.n_qt;
+      if (i == 1 && !has_b) continue;
       const int qt = i == 0 ? qa : qb;
-      const int row = (warp % 4) * 32 + lane;
-      const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
-      const uint32_t t_s = lane_addr + tm_s(i), t_o = lane_addr + tm_o(i);
-      const float sl2 = p.sl2;
       float m_run = -INFINITY, l_run = 0.f;
-      bool ok = true;
       for (int t = 0; t <= qt; ++t) {
-        ok = wait_bounded(&s_full[i], t & 1, abort_flag, p.err);
+        ok = wait_bounded(&s_full[i], s_phase, abort_flag, p.err);
+        s_phase ^= 1;
         if (!ok) break;
         tc_fence_after();
         uint32_t s0[64], s1[64];
         tmem_ld_x64(t_s, s0);
         tmem_ld_x64(t_s + 64, s1);
-        float x[128];
+        // diagonal tile: key column c is visible to row `row` iff c <= row
+        const int lim = (t == qt) ? row : 127;
+        float mx = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
-          x[c] = __uint_as_float(s0[c]) * sl2;
-          x[c + 64] = __uint_as_float(s1[c]) * sl2;
+          mx = fmaxf(mx, c <= lim ? __uint_as_float(s0[c]) : -INFINITY);
+          mx = fmaxf(mx, c + 64 <= lim ? __uint_as_float(s1[c]) : -INFINITY);
         }
-        if (t == qt) {  // diagonal tile: key column c is visible to row `row` iff c <= row
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c > row) x[c] = -INFINITY;
-        }
-        float mx = x[0];
-#pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
-        const float m_new = fmaxf(m_run, mx);
+        const float m_new = fmaxf(m_run, mx * sl2);
         const bool need = (m_new - m_run) > 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
-          if (need) m_run = m_new;
-          l_run *= alpha;
-          if (t > 0) {
-            // O_i was last written by PV_i(t-1), which completed before S_i(t) did.
-#pragma unroll
-            for (int c = 0; c < HD; c += 32) {
-              uint32_t r[32];
-              tmem_ld_x32(t_o + c, r);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-              tmem_st_x32(t_o + c, r);
-            }
-          }
-        }
+        const bool rescale = __any_sync(0xffffffffu, need);
+        const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
+        if (need) m_run = m_new;
+        l_run *= alpha;
+        const float neg_m = -m_run;
         float sum = 0.f;
-        uint32_t pk[64];
+        {
+          uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2_approx(x[2 * c] - m_run);
-          const float p1 = ex2_approx(x[2 * c + 1] - m_run);
-          sum += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = 2 * c <= lim ? ex2_approx(fmaf(__uint_as_float(s0[2 * c]), sl2, neg_m)) : 0.f;
+            const float p1 = 2 * c + 1 <= lim ? ex2_approx(fmaf(__uint_as_float(s0[2 * c + 1]), sl2, neg_m)) : 0.f;
+            sum += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_x32(t_s, pk);
+        }
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float p0 = 2 * c + 64 <= lim ? ex2_approx(fmaf(__uint_as_float(s1[2 * c]), sl2, neg_m)) : 0.f;
+            const float p1 =
+                2 * c + 65 <= lim ? ex2_approx(fmaf(__uint_as_float(s1[2 * c + 1]), sl2, neg_m)) : 0.f;
+            sum += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_x32(t_s + 32, pk);
         }
         l_run += sum;
-        tmem_st_x64(t_s, pk);
+        if (rescale && t > 0) {
+          // O_i was last written by PV_i(t-1), which completed before S_i(t) did.
+#pragma unroll
+          for (int c = 0; c < HD; c += 32) {
+            uint32_t r[32];
+            tmem_ld_x32(t_o + c, r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st_x32(t_o + c, r);
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_ready[i]);
       }
-      if (ok) ok = wait_bounded(&o_final[i], 0, abort_flag, p.err);
-      if (!ok) {
-        report_error(p.err, (K_FWD << 8) | SITE_SOFTMAX);
-        *abort_flag = 1;
-      } else {
-        // ---- epilogue: O row / l, stored at its original token; lse in natural log ----
-        tc_fence_after();
-        const int tok = tile_token0(qt) + row;
-        const float inv_l = 1.0f / l_run;
-        __nv_bfloat16* orow = p.o + ((size_t)(b * p.N + tok) * p.H + h) * HD;
+      if (ok) ok = wait_bounded(&o_final[i], o_items & 1, abort_flag, p.err);
+      if (!ok) break;
+      // ---- epilogue: O row / l, stored at its original token; lse in natural log ----
+      tc_fence_after();
+      const int tok = tile_token0(qt) + row;
+      const float inv_l = 1.0f / l_run;
+      __nv_bfloat16* orow = p.o + ((size_t)(b * p.N + tok) * p.H + h) * HD;
 #pragma unroll
-        for (int c = 0; c < HD; c += 32) {
-          uint32_t r[32];
-          tmem_ld_x32(t_o + c, r);
-          uint32_t pk[16];
+      for (int c = 0; c < HD; c += 32) {
+        uint32_t r[32];
+        tmem_ld_x32(t_o + c, r);
+        uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-        }
-        p.lse[((size_t)b * p.H + h) * p.N + tok] = (m_run + log2f(l_run)) * LN2;
+        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
+      p.lse[((size_t)b * p.H + h) * p.N + tok] = (m_run + log2f(l_run)) * LN2;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[i]);
+      ++o_items;
+    }
+    if (!ok) {
+      report_error(p.err, (K_FWD << 8) | SITE_SOFTMAX);
+      *abort_flag = 1;
     }
   }
 
@@ -354,7 +406,7 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
   p.n_groups = s.N / s.G;
   p.sl2 = (float)(1.4426950408889634 / sqrt((double)s.D));
   p.err = err;
-  const long long grid = (long long)p.n_pairs * s.B * s.H * p.n_groups;
+  const long long grid = (long long)((p.n_pairs + 1) / 2) * s.B * s.H * p.n_groups;
   if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(fwd::s2attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)fwd::SMEM_BYTES);

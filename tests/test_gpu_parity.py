@@ -156,7 +156,8 @@ def test_bf16_rejects_unsupported_shapes():
 def _sample_units(w):
     last = w.groups - 1
     shifted = w.H - 1
-    units = {(0, 0, 0), (0, 0, last), (0, shifted, last), (0, shifted, 0), (0, w.H - w.shift_heads, min(1, last))}
+    first_shifted = min(w.H - w.shift_heads, w.H - 1)
+    units = {(0, 0, 0), (0, 0, last), (0, shifted, last), (0, shifted, 0), (0, first_shifted, min(1, last))}
     return sorted(units)
 
 
