@@ -127,6 +127,31 @@ int s2attn_bwd_f32(const float* q, const float* k, const float* v, const float* 
 int rope_pi_apply(void* q, void* k, int B, int N, int H, int D, float pos_scale, float base, void* stream);
 
 /*
+ * Backward pass that allocates nothing.  The LongLoRA pages have no counterpart of
+ * this entry point; it exists for callers that cannot allocate device memory on
+ * the call path (a runtime whose allocator already holds the device's memory, a
+ * plugin whose enqueue step must not allocate, or a latency-critical loop that
+ * cannot afford cudaMalloc's implicit device synchronisation) and so cannot hand
+ * s2attn_bwd a workspace.
+ * Same arguments, shape rules and results as s2attn_bwd, minus the workspace: the
+ * fp32 dQ accumulator and delta live in a fixed array of
+ * S2ATTN_NOALLOC_SCRATCH_BYTES in the library's device memory, reserved on every
+ * device where the library's module is loaded and held until the process exits.
+ * Problems needing more (B*N*H*D*4 + B*H*N*4 bytes, each part rounded up to 256)
+ * return S2ATTN_ERR_WORKSPACE; at D = 128 that is about 130k (token, head) rows.
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream capture.
+ * Every call uses the same array and leaves its last contents there (the
+ * accumulator is zeroed at the start of each call): calls whose work overlaps on
+ * the GPU -- on different streams, or on different host threads -- race on it.
+ * Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define S2ATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                       const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int D, int G,
+                       int shift_heads, void* stream);
+
+/*
  * Reads the current device's error word: S2ATTN_OK if no kernel has failed since
  * the last clear, else S2ATTN_ERR_DEVICE_TIMEOUT with *detail (if non-NULL) set to
  * (kernel << 8) | site (kernel 1 = forward, 2 = backward).  Synchronize the streams

@@ -12,7 +12,7 @@ import os
 __all__ = [
     "S2AttnError", "capi", "library_path",
     "s2attn_fwd", "s2attn_bwd", "s2attn_bwd_workspace_bytes", "s2attn_bwd_preprocess", "s2attn_bwd_main",
-    "s2attn_bwd_dq_convert", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply",
+    "s2attn_bwd_dq_convert", "s2attn_bwd_noalloc", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply",
     "get_device_error", "clear_device_error",
 ]
 
@@ -51,6 +51,7 @@ def capi():
         "s2attn_bwd_preprocess": ([P, P, P, P, I, I, I, I, P], I),
         "s2attn_bwd_main": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P], I),
         "s2attn_bwd_dq_convert": ([P, P, I, I, I, I, P], I),
+        "s2attn_bwd_noalloc": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P], I),
         "s2attn_fwd_f32": ([P, P, P, P, P, I, I, I, I, I, I, P], I),
         "s2attn_bwd_f32": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, Z, P], I),
         "rope_pi_apply": ([P, P, I, I, I, I, F, F, P], I),
@@ -126,6 +127,16 @@ def s2attn_bwd_dq_convert(dq_acc, dq, stream=None):
     B, N, H, D = _bnhd(dq, "dq")
     _check("s2attn_bwd_dq_convert", capi().s2attn_bwd_dq_convert(_ptr(dq_acc), _ptr(dq), B, N, H, D,
                                                                  _stream(stream)))
+
+
+def s2attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, stream=None):
+    """bf16 backward without a caller workspace: for callers that cannot allocate device
+    memory.  Uses the library's fixed device scratch (S2ATTN_NOALLOC_SCRATCH_BYTES per
+    device, shared by all calls; overlapping calls race)."""
+    B, N, H, D = _bnhd(q, "q")
+    _check("s2attn_bwd_noalloc", capi().s2attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout),
+                                                           _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, D, G,
+                                                           shift_heads, _stream(stream)))
 
 
 def s2attn_fwd_f32(q, k, v, o, lse, G, shift_heads, stream=None):
