@@ -91,6 +91,48 @@ __device__ __forceinline__ void issue_pv(uint32_t d, uint32_t tp, uint32_t sv, u
   }
 }
 
+// P = exp2(s * sl2 - m) for one 128-column row of S, packed to bf16 pairs and written
+// over the first 64 TMEM columns of S.  Columns c > lim are masked (diagonal tile).
+// Returns the row sum of the fp32 P values (8 partial sums, no long dependency chain).
+template <bool MASK>
+__device__ __forceinline__ float softmax_p_row(const uint32_t (&s0)[64], const uint32_t (&s1)[64], int lim,
+                                               float sl2, float neg_m, uint32_t t_s) {
+  float sp[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) sp[e] = 0.f;
+  {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      float p0 = ex2_approx(fmaf(__uint_as_float(s0[2 * c]), sl2, neg_m));
+      float p1 = ex2_approx(fmaf(__uint_as_float(s0[2 * c + 1]), sl2, neg_m));
+      if (MASK) {
+        p0 = 2 * c <= lim ? p0 : 0.f;
+        p1 = 2 * c + 1 <= lim ? p1 : 0.f;
+      }
+      sp[c % 8] += p0 + p1;
+      pk[c] = pack_bf16x2(p0, p1);
+    }
+    tmem_st_x32(t_s, pk);
+  }
+  {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      float p0 = ex2_approx(fmaf(__uint_as_float(s1[2 * c]), sl2, neg_m));
+      float p1 = ex2_approx(fmaf(__uint_as_float(s1[2 * c + 1]), sl2, neg_m));
+      if (MASK) {
+        p0 = 2 * c + 64 <= lim ? p0 : 0.f;
+        p1 = 2 * c + 65 <= lim ? p1 : 0.f;
+      }
+      sp[c % 8] += p0 + p1;
+      pk[c] = pack_bf16x2(p0, p1);
+    }
+    tmem_st_x32(t_s + 32, pk);
+  }
+  return ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+}
+
 __global__ void __launch_bounds__(NTHREADS, 1)
     s2attn_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv, const Params p) {
@@ -296,12 +338,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_ld_x64(t_s + 64, s1);
         // diagonal tile: key column c is visible to row `row` iff c <= row
         const int lim = (t == qt) ? row : 127;
-        float mx = -INFINITY;
+        // row max: 8 independent partial maxima (a single chain would serialise 128 FMNMX)
+        float mxp[8];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          mx = fmaxf(mx, c <= lim ? __uint_as_float(s0[c]) : -INFINITY);
-          mx = fmaxf(mx, c + 64 <= lim ? __uint_as_float(s1[c]) : -INFINITY);
+        for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
+        if (t == qt) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            mxp[c % 8] = fmaxf(mxp[c % 8], c <= lim ? __uint_as_float(s0[c]) : -INFINITY);
+            mxp[c % 8] = fmaxf(mxp[c % 8], c + 64 <= lim ? __uint_as_float(s1[c]) : -INFINITY);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            mxp[c % 8] = fmaxf(mxp[c % 8], __uint_as_float(s0[c]));
+            mxp[c % 8] = fmaxf(mxp[c % 8], __uint_as_float(s1[c]));
+          }
         }
+        const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                               fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool need = (m_new - m_run) > 8.0f;
         const bool rescale = __any_sync(0xffffffffu, need);
@@ -309,30 +364,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (need) m_run = m_new;
         l_run *= alpha;
         const float neg_m = -m_run;
-        float sum = 0.f;
-        {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = 2 * c <= lim ? ex2_approx(fmaf(__uint_as_float(s0[2 * c]), sl2, neg_m)) : 0.f;
-            const float p1 = 2 * c + 1 <= lim ? ex2_approx(fmaf(__uint_as_float(s0[2 * c + 1]), sl2, neg_m)) : 0.f;
-            sum += p0 + p1;
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          tmem_st_x32(t_s, pk);
-        }
-        {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = 2 * c + 64 <= lim ? ex2_approx(fmaf(__uint_as_float(s1[2 * c]), sl2, neg_m)) : 0.f;
-            const float p1 =
-                2 * c + 65 <= lim ? ex2_approx(fmaf(__uint_as_float(s1[2 * c + 1]), sl2, neg_m)) : 0.f;
-            sum += p0 + p1;
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          tmem_st_x32(t_s + 32, pk);
-        }
+        const float sum = (t == qt) ? softmax_p_row<true>(s0, s1, lim, sl2, neg_m, t_s)
+                                    : softmax_p_row<false>(s0, s1, 127, sl2, neg_m, t_s);
         l_run += sum;
         if (rescale && t > 0) {
           // O_i was last written by PV_i(t-1), which completed before S_i(t) did.
