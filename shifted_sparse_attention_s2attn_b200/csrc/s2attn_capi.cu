@@ -149,15 +149,13 @@ int rope_table(int dev, int N, int D, float pos_scale, float base, RopeTable* ou
 
 int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout, const float* lse,
                   const float* delta, float* dq_acc, void* dk, void* dv, const s2::Shape& s, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  if (!map_bf16_sw128(&tq, q, s, 64) || !map_bf16_sw128(&tk, k, s, 128) || !map_bf16_sw128(&tv, v, s, 128) ||
-      !map_bf16_sw128(&tdo, dout, s, 64) ||
-      !make_map(&tdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, s.B, s.N, s.H, s.D, 128, 64,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
+  CUtensorMap tq, tk, tv, tdo;
+  if (!map_bf16_sw128(&tq, q, s, 128) || !map_bf16_sw128(&tk, k, s, 128) || !map_bf16_sw128(&tv, v, s, 128) ||
+      !map_bf16_sw128(&tdo, dout, s, 128))
     return S2ATTN_ERR_CUDA;
   int* err = error_word_ptr();
   if (!err) return S2ATTN_ERR_CUDA;
-  return cuda_status(s2::launch_bwd_sm100(tq, tk, tv, tdo, tdq, lse, delta, dk, dv, s, err, st));
+  return cuda_status(s2::launch_bwd_sm100(tq, tk, tv, tdo, lse, delta, dq_acc, dk, dv, s, err, st));
 }
 
 }  // namespace
