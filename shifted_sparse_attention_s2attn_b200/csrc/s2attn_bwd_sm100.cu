@@ -10,6 +10,9 @@
 // token (r + G/2) mod N, and every 128-row tile of rolled rows is a contiguous run of
 // original rows, so TMA boxes and stores address the original tensors directly.
 //
+// Shared memory: K, V; a 3-stage Q (+ lse) ring and a 2-stage dO (+ delta) ring; once
+// dP(g) is complete dO(g) is dead, and its slot receives dS^T(g) for dK(g) and dQ(g).
+//
 // Work item: (b, h, group j, key tile kt of 128 keys).  The CTA keeps K and V in
 // shared memory and walks the query tiles of the group that can see these keys
 // (tiles kt .. G/128-1), computing per tile
@@ -28,14 +31,14 @@
 //   dV(g) | dP(g) [after dQ(g-1) was drained] | S(g+1) | dK(g), dQ(g)
 // so S(g+1) overlaps the dS work and dV(g+1) overlaps the dQ(g) drain.
 //
-// Warp roles (448 threads, <= 128 registers each):
+// Warp roles (512 threads; registers rebalanced with setmaxnreg, see REGS_*):
 //   warps 0-3, 4-7  P / dS, thread = key row (TMEM lane); warpgroup w takes query
 //                   columns [64w, 64w+64) of each tile: P^T to TMEM (bf16), dS^T to
 //                   a 128-byte-swizzled smem tile; at the end of an item warpgroup 0
 //                   stores dK and warpgroup 1 stores dV
 //   warps 8-11      dQ drain: thread = head dim d; dQ^T from TMEM, one coalesced
 //                   fp32 reduction per (query, warp) into the global accumulator
-//   warp  12        TMA producer (K, V per item; Q, dO, lse, delta through a 2-stage ring)
+//   warp  12        TMA producer (K, V per item; Q + lse and dO + delta through rings)
 //   warp  13        MMA issuer
 #include "s2_internal.h"
 #include "s2_ptx.cuh"
@@ -48,20 +51,25 @@ constexpr int BQ = 128;  // queries per tile
 constexpr int HD = 128;
 constexpr uint32_t BOX = 128 * 128;        // 128 rows x 128 B (64 bf16 columns)
 constexpr uint32_t TILE = 2 * BOX;         // 128 rows x 128 bf16 = 32 KB
-constexpr int QSTAGES = 2;
+// Q (+ lse) ring of 3 tiles, dO (+ delta) ring of 2.  Once dP(g) has completed, dO(g) is
+// dead and its slot receives dS^T(g) (2 boxes: queries 0-63, 64-127), read by dK(g), dQ(g).
+constexpr int QSTAGES = 3, DSTAGES = 2;
 constexpr uint32_t OFF_K = 0;
 constexpr uint32_t OFF_V = TILE;
 constexpr uint32_t OFF_Q = 2 * TILE;                   // [QSTAGES] tiles
-constexpr uint32_t OFF_DO = OFF_Q + QSTAGES * TILE;    // [QSTAGES] tiles
-constexpr uint32_t OFF_DS = OFF_DO + QSTAGES * TILE;   // dS^T: 2 boxes (queries 0-63, 64-127)
-constexpr uint32_t OFF_STAT = OFF_DS + TILE;           // [QSTAGES] x (lse[128], delta[128]) fp32
-constexpr uint32_t STAT_BYTES = 2 * BQ * 4;
-constexpr uint32_t OFF_BAR = OFF_STAT + QSTAGES * STAT_BYTES;
-constexpr int NBARS = 18;
+constexpr uint32_t OFF_DO = OFF_Q + QSTAGES * TILE;    // [DSTAGES] tiles (dO, then dS^T)
+constexpr uint32_t OFF_LSE = OFF_DO + DSTAGES * TILE;  // [QSTAGES] x lse[128] fp32
+constexpr uint32_t OFF_DELTA = OFF_LSE + QSTAGES * BQ * 4;  // [DSTAGES] x delta[128] fp32
+constexpr uint32_t OFF_BAR = OFF_DELTA + DSTAGES * BQ * 4;
+constexpr int NBARS = 21;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;  // the dynamic smem base must be 1024-byte aligned
-constexpr int NTHREADS = 448;
+constexpr int NTHREADS = 512;  // warpgroups: P/dS, P/dS, dQ drain, producer + MMA (+2 idle warps)
 constexpr int WARP_DQ0 = 8, WARP_LOAD = 12, WARP_MMA = 13;
+// Launch: 512 threads x 128 registers = 65536.  After setmaxnreg: P/dS warpgroups keep 128,
+// the dQ drain gets 168 (it holds a whole 128-column dQ^T row), producer/MMA drop to 88:
+// 2 x 128 x 128 + 128 x 168 + 128 x 88 = 65536.
+constexpr int REGS_DRAIN = 168, REGS_CONTROL = 88;
 constexpr uint32_t PDS_WARPS = 8;
 
 constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DK = 256, TM_DV = 384;
@@ -121,18 +129,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* q_full = bars + 2;     // [2]
-  uint64_t* q_empty = bars + 4;    // [2]
-  uint64_t* s_full = bars + 6;
-  uint64_t* p_ready = bars + 7;
-  uint64_t* dp_full = bars + 8;
-  uint64_t* ds_ready = bars + 9;
-  uint64_t* ds_free = bars + 10;
-  uint64_t* dq_full = bars + 11;
-  uint64_t* dq_free = bars + 12;
-  uint64_t* mma_done = bars + 13;
-  uint64_t* dkv_empty = bars + 14;
-  uint64_t* drain = bars + 15;
+  uint64_t* q_full = bars + 2;     // [3]
+  uint64_t* q_empty = bars + 5;    // [3]
+  uint64_t* do_full = bars + 8;    // [2]
+  uint64_t* do_empty = bars + 10;  // [2]
+  uint64_t* s_full = bars + 12;
+  uint64_t* p_ready = bars + 13;
+  uint64_t* dp_full = bars + 14;
+  uint64_t* ds_ready = bars + 15;
+  uint64_t* dq_full = bars + 16;
+  uint64_t* dq_free = bars + 17;
+  uint64_t* mma_done = bars + 18;
+  uint64_t* dkv_empty = bars + 19;
+  uint64_t* drain = bars + 20;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -169,11 +178,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
     }
+    for (int s = 0; s < DSTAGES; ++s) {
+      mbar_init(&do_full[s], 1);
+      mbar_init(&do_empty[s], 1);
+    }
     mbar_init(s_full, 1);
     mbar_init(p_ready, PDS_WARPS);
     mbar_init(dp_full, 1);
     mbar_init(ds_ready, PDS_WARPS);
-    mbar_init(ds_free, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 4);
     mbar_init(mma_done, 1);
@@ -191,8 +203,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool skip = *abort_flag != 0;
+  const int wg = __shfl_sync(0xffffffffu, (int)threadIdx.x / 128, 0);  // warp-uniform warpgroup index
 
-  if (!skip && warp == WARP_LOAD && lane == 0) {
+  // setmaxnreg must dominate the code that relies on the new register budget
+  if (wg == 3) {
+   regs_dec<REGS_CONTROL>();
+   if (!skip && warp == WARP_LOAD && lane == 0) {
     // ---------------- TMA producer ----------------
     prefetch_tmap(&tq);
     prefetch_tmap(&tk);
@@ -201,7 +217,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     const int row_base = b * p.N;
     const size_t stat_base = ((size_t)b * p.H + h) * p.N;
-    int kv_loads = 0, q_armed = 0;
+    int kv_loads = 0, q_armed = 0, do_armed = 0;
     for (int it = 0; it < n_items && ok; ++it) {
       const int kt = kts[it];
       if (it > 0) {
@@ -218,18 +234,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int nsteps = steps_of(kt);
       for (int s = 0; s < nsteps; ++s) {
         const int g = q_armed;
-        const int st = g % QSTAGES;
-        ok = wait_bounded(&q_empty[st], ((g / QSTAGES) & 1) ^ 1, abort_flag, p.err);
-        if (!ok) break;
         const int tok = token_of((kt + s) * BQ);
-        mbar_arrive_expect_tx(&q_full[st], 2 * TILE + STAT_BYTES);
-        for (int x = 0; x < 2; ++x) {
-          tma_load_3d(smem + OFF_Q + st * TILE + x * BOX, &tq, x * 64, h, row_base + tok, &q_full[st]);
-          tma_load_3d(smem + OFF_DO + st * TILE + x * BOX, &tdo, x * 64, h, row_base + tok, &q_full[st]);
-        }
-        bulk_load(smem + OFF_STAT + st * STAT_BYTES, p.lse + stat_base + tok, BQ * 4, &q_full[st]);
-        bulk_load(smem + OFF_STAT + st * STAT_BYTES + BQ * 4, p.delta + stat_base + tok, BQ * 4, &q_full[st]);
+        const int qs = g % QSTAGES, ds = g % DSTAGES;
+        ok = wait_bounded(&q_empty[qs], ((g / QSTAGES) & 1) ^ 1, abort_flag, p.err);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&q_full[qs], TILE + BQ * 4);
+        for (int x = 0; x < 2; ++x)
+          tma_load_3d(smem + OFF_Q + qs * TILE + x * BOX, &tq, x * 64, h, row_base + tok, &q_full[qs]);
+        bulk_load(smem + OFF_LSE + qs * BQ * 4, p.lse + stat_base + tok, BQ * 4, &q_full[qs]);
         q_armed = g + 1;
+        ok = wait_bounded(&do_empty[ds], ((g / DSTAGES) & 1) ^ 1, abort_flag, p.err);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&do_full[ds], TILE + BQ * 4);
+        for (int x = 0; x < 2; ++x)
+          tma_load_3d(smem + OFF_DO + ds * TILE + x * BOX, &tdo, x * 64, h, row_base + tok, &do_full[ds]);
+        bulk_load(smem + OFF_DELTA + ds * BQ * 4, p.delta + stat_base + tok, BQ * 4, &do_full[ds]);
+        do_armed = g + 1;
       }
     }
     if (!ok) {
@@ -239,49 +259,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool dok = kv_loads == 0 || wait_drain(kv_full, (kv_loads - 1) & 1);
     for (int g = (q_armed > QSTAGES ? q_armed - QSTAGES : 0); g < q_armed; ++g)
       dok &= wait_drain(&q_full[g % QSTAGES], (g / QSTAGES) & 1);
+    for (int g = (do_armed > DSTAGES ? do_armed - DSTAGES : 0); g < do_armed; ++g)
+      dok &= wait_drain(&do_full[g % DSTAGES], (g / DSTAGES) & 1);
     if (!dok) report_error(p.err, (K_BWD << 8) | SITE_DRAIN);
-  } else if (!skip && warp == WARP_MMA && lane == 0) {
+   } else if (!skip && warp == WARP_MMA && lane == 0) {
     // ---------------- MMA issuer ----------------
     const uint32_t id_kq = idesc_bf16_f32(BK, BQ, false, false);   // S^T, dP^T
     const uint32_t id_dkv = idesc_bf16_f32(BK, HD, false, true);   // dV (A = P^T in TMEM), dK (A = dS^T)
     const uint32_t id_dq = idesc_bf16_f32(HD, BQ, true, true);     // dQ^T = K^T dS^T
     const uint32_t sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
-    const uint32_t sq0 = smem_u32(smem + OFF_Q), sdo0 = smem_u32(smem + OFF_DO), sds = smem_u32(smem + OFF_DS);
+    const uint32_t sq0 = smem_u32(smem + OFF_Q), sdo0 = smem_u32(smem + OFF_DO);
     bool ok = true;
     int g0 = 0;  // global index of the current item's first query tile
     for (int it = 0; it < n_items && ok; ++it) {
       const int nsteps = steps_of(kts[it]);
-      // prologue: S(g0) and dP(g0); dP^T's columns last held dQ^T(g0-1)
+      // prologue: S(g0)
       ok = wait_bounded(kv_full, it & 1, abort_flag, p.err);
       if (ok) ok = wait_bounded(&q_full[g0 % QSTAGES], (g0 / QSTAGES) & 1, abort_flag, p.err);
-      if (ok && g0 > 0) ok = wait_bounded(dq_free, (g0 - 1) & 1, abort_flag, p.err);
       if (!ok) break;
       tc_fence_after();
       issue_kq(tmem + TM_S, sk, sq0 + (g0 % QSTAGES) * TILE, id_kq);
       mma_commit(s_full);
-      issue_kq(tmem + TM_DP, sv, sdo0 + (g0 % QSTAGES) * TILE, id_kq);
-      mma_commit(dp_full);
       for (int s = 0; s < nsteps && ok; ++s) {
         const int g = g0 + s;
-        const int st = g % QSTAGES;
-        const uint32_t sq = sq0 + st * TILE, sdo = sdo0 + st * TILE;
+        const uint32_t sq = sq0 + (g % QSTAGES) * TILE;
+        const uint32_t sdo = sdo0 + (g % DSTAGES) * TILE;  // dO(g), later dS^T(g)
         // dV += P^T dO
-        ok = wait_bounded(p_ready, g & 1, abort_flag, p.err);
+        ok = wait_bounded(&do_full[g % DSTAGES], (g / DSTAGES) & 1, abort_flag, p.err);
+        if (ok) ok = wait_bounded(p_ready, g & 1, abort_flag, p.err);
         if (ok && s == 0 && it > 0) ok = wait_bounded(dkv_empty, (it - 1) & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk)
-          mma_ts(tmem + TM_DV, tmem + TM_S + (kk / 4) * 64 + (kk % 4) * 8,
-                 sdesc_sw128(sdo + (kk / 8) * BOX + (kk % 8) * 2048, BOX, 1024), id_dkv, (s > 0 || kk > 0) ? 1u : 0u);
-        // dP(g) once dQ^T(g-1) has left the shared columns
-        if (s > 0) {
-          ok = wait_bounded(dq_free, (g - 1) & 1, abort_flag, p.err);
-          if (!ok) break;
-          tc_fence_after();
-          issue_kq(tmem + TM_DP, sv, sdo, id_kq);
-          mma_commit(dp_full);
-        }
+          mma_ts(tmem + TM_DV, tmem + TM_S + (kk / 4) * 64 + (kk % 4) * 8, sdesc_sw128(sdo + kk * 2048, BOX, 1024),
+                 id_dkv, (s > 0 || kk > 0) ? 1u : 0u);
+        // dP(g) once dQ^T(g-1) has left the shared columns.  Always issued after dV(g):
+        // its completion (dp_full) then also means dV(g) has finished reading dO(g),
+        // whose slot the dS warps overwrite with dS^T(g).
+        if (g > 0) ok = wait_bounded(dq_free, (g - 1) & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        issue_kq(tmem + TM_DP, sv, sdo, id_kq);
+        mma_commit(dp_full);
         // S(g+1): its columns held P^T(g), read by the dV MMAs above (issued first)
         if (s + 1 < nsteps) {
           ok = wait_bounded(&q_full[(g + 1) % QSTAGES], ((g + 1) / QSTAGES) & 1, abort_flag, p.err);
@@ -296,15 +316,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk)
-          mma_ss(tmem + TM_DK, sdesc_sw128(sds + (kk / 4) * BOX + (kk % 4) * 32, 16, 1024),
-                 sdesc_sw128(sq + (kk / 8) * BOX + (kk % 8) * 2048, BOX, 1024), id_dkv, (s > 0 || kk > 0) ? 1u : 0u);
+          mma_ss(tmem + TM_DK, sdesc_sw128(sdo + (kk / 4) * BOX + (kk % 4) * 32, 16, 1024),
+                 sdesc_sw128(sq + kk * 2048, BOX, 1024), id_dkv, (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
-          mma_ss(tmem + TM_DP, sdesc_sw128(sk + kk * 2048, BOX, 1024), sdesc_sw128(sds + kk * 2048, BOX, 1024),
+          mma_ss(tmem + TM_DP, sdesc_sw128(sk + kk * 2048, BOX, 1024), sdesc_sw128(sdo + kk * 2048, BOX, 1024),
                  id_dq, kk > 0 ? 1u : 0u);
         mma_commit(dq_full);
-        mma_commit(ds_free);
-        mma_commit(&q_empty[st]);
+        mma_commit(&q_empty[g % QSTAGES]);   // Q(g) and dS^T(g) (in the dO slot) no longer read
+        mma_commit(&do_empty[g % DSTAGES]);
       }
       if (!ok) break;
       mma_commit(mma_done);  // dK, dV of this item complete
@@ -317,7 +337,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     mma_commit(drain);
     if (!wait_drain(drain, 0)) report_error(p.err, (K_BWD << 8) | SITE_DRAIN);
-  } else if (!skip && warp < 8) {
+   }
+  } else if (wg < 2) {
+   if (!skip) {
     // ---------------- P / dS warps: thread = key row, 64 query columns per warpgroup ----------------
     const int hf = warp / 4;
     const int kr = (warp % 4) * 32 + lane;
@@ -329,10 +351,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int kt = kts[it];
       const int nsteps = steps_of(kt);
       for (int s = 0; s < nsteps; ++s, ++g) {
-        const int st = g % QSTAGES;
-        const float* lse_s = reinterpret_cast<const float*>(smem + OFF_STAT + st * STAT_BYTES) + 64 * hf;
-        const float* delta_s = reinterpret_cast<const float*>(smem + OFF_STAT + st * STAT_BYTES + BQ * 4) + 64 * hf;
-        ok = wait_bounded(&q_full[st], (g / QSTAGES) & 1, abort_flag, p.err);
+        const float* lse_s = reinterpret_cast<const float*>(smem + OFF_LSE + (g % QSTAGES) * BQ * 4) + 64 * hf;
+        const float* delta_s = reinterpret_cast<const float*>(smem + OFF_DELTA + (g % DSTAGES) * BQ * 4) + 64 * hf;
+        ok = wait_bounded(&q_full[g % QSTAGES], (g / QSTAGES) & 1, abort_flag, p.err);
         if (ok) ok = wait_bounded(s_full, g & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
@@ -366,17 +387,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(p_ready);
 
-        ok = wait_bounded(dp_full, g & 1, abort_flag, p.err);
-        if (ok && g > 0) ok = wait_bounded(ds_free, (g - 1) & 1, abort_flag, p.err);
+        // dP(g) complete => every earlier MMA (dV(g) included) is too: dO(g) is dead and
+        // its slot takes dS^T(g)
+        ok = wait_bounded(&do_full[g % DSTAGES], (g / DSTAGES) & 1, abort_flag, p.err);
+        if (ok) ok = wait_bounded(dp_full, g & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
         // dS^T row kr: this warpgroup's 64 queries = box hf, one 128-byte row of 8 chunks;
         // chunk c is stored at chunk slot c ^ (kr % 8) (128-byte swizzle)
-        uint8_t* dsrow = smem + OFF_DS + hf * BOX + kr * 128;
+        uint8_t* dsrow = smem + OFF_DO + (g % DSTAGES) * TILE + hf * BOX + kr * 128;
+        uint32_t dr0[32], dr1[32];
+        tmem_ld_x32_nowait(lane_addr + TM_DP + 64 * hf, dr0);
+        tmem_ld_x32_nowait(lane_addr + TM_DP + 64 * hf + 32, dr1);
+        tmem_wait_ld_x32(dr0);
+        tmem_mark_loaded_x32(dr1);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t dr[32];
-          tmem_ld_x32(lane_addr + TM_DP + 64 * hf + 32 * half, dr);
+          const uint32_t* dr = half == 0 ? dr0 : dr1;
           uint32_t pk[16];
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
@@ -414,7 +441,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       report_error(p.err, (K_BWD << 8) | SITE_PDS);
       *abort_flag = 1;
     }
-  } else if (!skip && warp >= WARP_DQ0 && warp < WARP_DQ0 + 4) {
+   }
+  } else {
+   regs_inc<REGS_DRAIN>();
+   if (!skip) {
     // ---------------- dQ drain: thread = head dim d ----------------
     const int d = (warp - WARP_DQ0) * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
@@ -430,17 +460,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // query q of this tile -> dq_acc[b, tok0 + q, h, d]; a warp covers 32 consecutive d (128 B)
         float* dst = p.dq_acc + ((size_t)(b * p.N + token_of((kt + s) * BQ)) * p.H + h) * HD + d;
         const size_t row_stride = (size_t)p.H * HD;
-#pragma unroll 1
-        for (int c = 0; c < BQ; c += 32) {
-          uint32_t r[32];
-          tmem_ld_x32(lane_addr + TM_DP + c, r);
-          if (c + 32 == BQ) {  // all of dQ^T(g) is in registers: release the columns
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(dq_free);
-          }
+        uint32_t r0[64], r1[64];
+        tmem_ld_x64(lane_addr + TM_DP, r0);
+        tmem_ld_x64(lane_addr + TM_DP + 64, r1);
+        // all of dQ^T(g) is in registers: release the columns before the reductions
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free);
+        // one running address (consecutive queries are row_stride floats apart)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) red_add_f32(dst + (size_t)(c + e) * row_stride, __uint_as_float(r[e]));
+        for (int e = 0; e < 64; ++e) {
+          red_add_f32(dst, __uint_as_float(r0[e]));
+          dst += row_stride;
+        }
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          red_add_f32(dst, __uint_as_float(r1[e]));
+          dst += row_stride;
         }
       }
     }
@@ -448,6 +484,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       report_error(p.err, (K_BWD << 8) | SITE_DQ);
       *abort_flag = 1;
     }
+   }
   }
 
   tc_fence_before();

@@ -75,20 +75,23 @@ struct Params {
 
 enum Site : int { SITE_LOAD = 1, SITE_MMA = 2, SITE_SOFTMAX = 3, SITE_EPILOGUE = 4, SITE_DRAIN = 5 };
 
+// Descriptors are built once per GEMM and stepped by constant offsets, so each MMA
+// costs the issuing thread (which shares its SM sub-partition with softmax warps) only
+// a few instructions.
 __device__ __forceinline__ void issue_s(uint32_t d, uint32_t sq, uint32_t sk, uint32_t idesc) {
+  const uint64_t dq = sdesc_sw128(sq, 16, 1024), dk = sdesc_sw128(sk, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
     const uint32_t off = (kk / 4) * BOX_BYTES + (kk % 4) * 32;
-    mma_ss(d, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+    mma_ss(d, sdesc_add(dq, off), sdesc_add(dk, off), idesc, kk > 0 ? 1u : 0u);
   }
 }
 
 __device__ __forceinline__ void issue_pv(uint32_t d, uint32_t tp, uint32_t sv, uint32_t idesc, bool first) {
+  // B = V^T viewed MN-major: 16 key rows (2 KB) per k-step, 64-column boxes BOX_BYTES apart.
+  const uint64_t dv = sdesc_sw128(sv, BOX_BYTES, 1024);
 #pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk) {
-    // B = V^T viewed MN-major: 16 key rows (2 KB) per k-step, 64-column boxes BOX_BYTES apart.
-    mma_ts(d, tp + kk * 8, sdesc_sw128(sv + kk * 2048, BOX_BYTES, 1024), idesc, (first && kk == 0) ? 0u : 1u);
-  }
+  for (int kk = 0; kk < BN / 16; ++kk) mma_ts(d, tp + kk * 8, sdesc_add(dv, kk * 2048), idesc, (first && kk == 0) ? 0u : 1u);
 }
 
 // P = exp2(s * sl2 - m) for one 128-column row of S, packed to bf16 pairs and written
