@@ -45,6 +45,21 @@ def step_flops(w):
     return 3.5 * 4 * w.D * useful_pairs(w)
 
 
+def max_over_ranks(ms, device=None):
+    """Slowest rank's time: every rank contributes its own CUDA-event time (replicas)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_step, steps, world, ms_max):
+    """Work of all ranks (world replicas x steps x FLOPs per step) over the slowest rank's time."""
+    return world * flops_per_step * steps / (ms_max / 1e3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -293,10 +308,7 @@ def run_ours(args, w):
     if rc != 0:
         raise SystemExit(f"device error word set during the timed region: {detail:#x}")
 
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dev)
 
     # ---- end to end: host buffers in, results out, through the same public calls ----
     e2e_steps = max(3, min(args.steps, 10))
@@ -324,17 +336,14 @@ def run_ours(args, w):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
     flops = step_flops(w)
-    value = world * flops * args.steps / (ms_max / 1e3) / 1e12
+    value = whole_job_tflops(flops, args.steps, world, ms_max)
     peaks, peak_src = load_peaks()
     fwd_flops, bwd_flops = 4 * D * useful_pairs(w), 10 * D * useful_pairs(w)
     bwd_avg = statistics.mean(bwd_ms) / 1e3
@@ -358,7 +367,7 @@ def run_ours(args, w):
                          "achieved": fwd_flops / fwd_avg / 1e12, "peak": peak_sus, "unit": "TFLOP/s",
                          "frac": fwd_flops / fwd_avg / 1e12 / peak_sus,
                          "traffic": traffic_record("s2attn_fwd_sm100.cu", "s2attn_fwd_kernel")},
-        "e2e": {"value": world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": whole_job_tflops(flops, e2e_steps, world, e2e_ms), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks,

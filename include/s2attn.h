@@ -162,6 +162,16 @@ int s2attn_get_device_error(int* detail);
 /* Resets the current device's error word to 0 (synchronous). */
 int s2attn_clear_device_error(void);
 
+/*
+ * Self-test of the device-side failure path used by every kernel above: launches one
+ * thread that waits on a barrier nothing ever arrives at, with a wait limit of
+ * `timeout_us` microseconds (1 .. 1000000).  After the caller synchronizes `stream`,
+ * s2attn_get_device_error() returns S2ATTN_ERR_DEVICE_TIMEOUT with detail
+ * (3 << 8) | 1, and the context stays usable (clear the word to continue).  The
+ * kernels' own waits give up after 2 s the same way instead of hanging the GPU.
+ */
+int s2attn_selftest_bounded_wait(unsigned timeout_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -13,7 +13,7 @@ __all__ = [
     "S2AttnError", "capi", "library_path",
     "s2attn_fwd", "s2attn_bwd", "s2attn_bwd_workspace_bytes", "s2attn_bwd_preprocess", "s2attn_bwd_main",
     "s2attn_bwd_dq_convert", "s2attn_bwd_noalloc", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply",
-    "get_device_error", "clear_device_error",
+    "get_device_error", "clear_device_error", "s2attn_selftest_bounded_wait",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -57,6 +57,7 @@ def capi():
         "rope_pi_apply": ([P, P, I, I, I, I, F, F, P], I),
         "s2attn_get_device_error": ([ctypes.POINTER(I)], I),
         "s2attn_clear_device_error": ([], I),
+        "s2attn_selftest_bounded_wait": ([ctypes.c_uint, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -170,3 +171,8 @@ def get_device_error():
 
 def clear_device_error():
     _check("s2attn_clear_device_error", capi().s2attn_clear_device_error())
+
+
+def s2attn_selftest_bounded_wait(timeout_us, stream=None):
+    """Runs a kernel whose bounded wait must time out (see include/s2attn.h)."""
+    _check("s2attn_selftest_bounded_wait", capi().s2attn_selftest_bounded_wait(int(timeout_us), _stream(stream)))

@@ -10,7 +10,7 @@ namespace s2 {
 
 // Device error codes (first failure wins; read with s2attn_get_device_error).
 // code = (kernel << 8) | site
-enum Kernel : int { K_FWD = 1, K_BWD = 2 };
+enum Kernel : int { K_FWD = 1, K_BWD = 2, K_SELFTEST = 3 };
 
 // Problem description after validation.  Rows of a [B,N,H,D] tensor for head h
 // are addressed through 3-D tensor maps with dims {D, H, B*N}.

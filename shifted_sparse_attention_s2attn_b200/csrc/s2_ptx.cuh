@@ -49,18 +49,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase of `bar` with the given parity.  Returns false if the
-// wait timed out, another role of this CTA raised *abort, or any CTA of the launch
-// already reported an error in the global error word *gerr.
-__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                             const int* gerr) {
+// Waits for the phase of `bar` with the given parity.  Returns false if the wait
+// outlasted `timeout_ns`, another role of this CTA raised *abort, or any CTA of the
+// launch already reported an error in the global error word *gerr.
+__device__ __forceinline__ bool wait_bounded_ns(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                const int* gerr, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort || *(const volatile int*)gerr) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
   }
+}
+
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                             const int* gerr) {
+  return wait_bounded_ns(bar, parity, abort, gerr, kWaitTimeoutNs);
 }
 
 // Teardown wait for copies or MMAs this thread itself started: only the time

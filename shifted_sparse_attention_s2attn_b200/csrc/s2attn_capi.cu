@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "s2_internal.h"
+#include "s2_ptx.cuh"
 #include "s2attn.h"
 
 namespace {
@@ -145,6 +146,21 @@ int rope_table(int dev, int N, int D, float pos_scale, float base, RopeTable* ou
   cache[key] = tab;
   *out = tab;
   return S2ATTN_OK;
+}
+
+// One thread waits on an mbarrier that nothing ever arrives at; the bounded wait must
+// give up after timeout_ns and record (K_SELFTEST << 8) | 1 in the error word.
+__global__ void selftest_wait_kernel(int* err, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    s2::mbar_init(&bar, 1);
+    abort_flag = 0;
+    s2::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !s2::wait_bounded_ns(&bar, 0, &abort_flag, err, timeout_ns))
+    s2::report_error(err, (s2::K_SELFTEST << 8) | 1);
 }
 
 int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout, const float* lse,
@@ -289,6 +305,14 @@ int rope_pi_apply(void* q, void* k, int B, int N, int H, int D, float pos_scale,
   if (rc) return rc;
   return cuda_status(
       s2::launch_rope_pi(q, k, tab.cos_d, tab.sin_d, B, N, H, D, static_cast<cudaStream_t>(stream)));
+}
+
+int s2attn_selftest_bounded_wait(unsigned timeout_us, void* stream) {
+  if (timeout_us == 0 || timeout_us > 1000000u) return S2ATTN_ERR_INVALID_ARG;
+  int* err = error_word_ptr();
+  if (!err) return S2ATTN_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, 1000ull * timeout_us);
+  return cuda_status(cudaGetLastError());
 }
 
 int s2attn_get_device_error(int* detail) {
