@@ -49,15 +49,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread may sleep in hardware until the phase
+// completes or about `hint_ns` have passed, instead of spinning.  Spinning waiters
+// flood the memory-instruction path that tcgen05.mma issue also uses.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity.  Returns false if the wait
 // outlasted `timeout_ns`, another role of this CTA raised *abort, or any CTA of the
-// launch already reported an error in the global error word *gerr.
+// launch already reported an error in the global error word *gerr.  The flags are
+// only looked at between hardware sleeps.
 __device__ __forceinline__ bool wait_bounded_ns(uint64_t* bar, uint32_t parity, volatile int* abort,
                                                 const int* gerr, uint64_t timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     if (*abort || *(const volatile int*)gerr) return false;
     if (globaltimer_ns() - t0 > timeout_ns) return false;
   }
@@ -74,7 +90,7 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
     if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
   }
 }
