@@ -28,8 +28,8 @@
 // pairs over columns [64w, 64w+32); dP^T [128,256), which dQ^T reuses once the dS warps have read dP^T;
 // dK [256,384); dV [384,512).
 // MMA issue order per query tile g (one thread; tcgen05 MMAs execute in issue order):
-//   dV(g) | dP(g) [after dQ(g-1) was drained] | S(g+1) | dK(g), dQ(g)
-// so S(g+1) overlaps the dS work and dV(g+1) overlaps the dQ(g) drain.
+//   dV(g) | dP(g) [after dQ(g-1) was drained] | S(g+1) | dQ(g), dK(g)
+// so S(g+1) overlaps the dS work and dK(g), dV(g+1) overlap the dQ(g) drain.
 //
 // Warp roles (512 threads; registers rebalanced with setmaxnreg, see REGS_*):
 //   warps 0-3, 4-7  P / dS, thread = key row (TMEM lane); warpgroup w takes query
@@ -111,10 +111,6 @@ __device__ __forceinline__ void store_row_bf16(uint32_t taddr, __nv_bfloat16* ds
 #pragma unroll
     for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
   }
-}
-
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
-  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }
 
 __device__ __forceinline__ void red_add_f32(float* addr, float v) {
@@ -264,11 +260,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!dok) report_error(p.err, (K_BWD << 8) | SITE_DRAIN);
    } else if (!skip && warp == WARP_MMA && lane == 0) {
     // ---------------- MMA issuer ----------------
+    // Each group of 8 MMAs blocks this thread until it is nearly all dispatched, so a
+    // barrier check that resolves only after the previous group leaves a bubble in the
+    // tensor pipe.  The barriers of each sync point are therefore probed (non-blocking)
+    // before the group ahead of it is issued; a blocking wait follows only if the probe
+    // found them incomplete.  Sync points per query tile g:
+    //   A: dO(g) loaded, P^T(g) in TMEM (item start: previous dK/dV read out)  -> dV(g)
+    //   B: dQ^T(g-1) drained from the shared columns                            -> dP(g)
+    //   C: Q(g+1) loaded                                                         -> S(g+1)
+    //   D: dS^T(g) in smem                                                       -> dQ(g), dK(g)
     const uint32_t id_kq = idesc_bf16_f32(BK, BQ, false, false);   // S^T, dP^T
     const uint32_t id_dkv = idesc_bf16_f32(BK, HD, false, true);   // dV (A = P^T in TMEM), dK (A = dS^T)
     const uint32_t id_dq = idesc_bf16_f32(HD, BQ, true, true);     // dQ^T = K^T dS^T
     const uint32_t sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
     const uint32_t sq0 = smem_u32(smem + OFF_Q), sdo0 = smem_u32(smem + OFF_DO);
+    auto ready_a = [&](int g, int it, int s, bool block) -> bool {
+      const bool need_empty = s == 0 && it > 0;
+      if (!block)
+        return mbar_test_wait(&do_full[g % DSTAGES], (g / DSTAGES) & 1) && mbar_test_wait(p_ready, g & 1) &&
+               (!need_empty || mbar_test_wait(dkv_empty, (it - 1) & 1));
+      return wait_bounded(&do_full[g % DSTAGES], (g / DSTAGES) & 1, abort_flag, p.err) &&
+             wait_bounded(p_ready, g & 1, abort_flag, p.err) &&
+             (!need_empty || wait_bounded(dkv_empty, (it - 1) & 1, abort_flag, p.err));
+    };
     bool ok = true;
     int g0 = 0;  // global index of the current item's first query tile
     for (int it = 0; it < n_items && ok; ++it) {
@@ -280,49 +294,63 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       issue_kq(tmem + TM_S, sk, sq0 + (g0 % QSTAGES) * TILE, id_kq);
       mma_commit(s_full);
+      bool pre_a = false;
       for (int s = 0; s < nsteps && ok; ++s) {
         const int g = g0 + s;
+        const bool next = s + 1 < nsteps;
         const uint32_t sq = sq0 + (g % QSTAGES) * TILE;
         const uint32_t sdo = sdo0 + (g % DSTAGES) * TILE;  // dO(g), later dS^T(g)
-        // dV += P^T dO
-        ok = wait_bounded(&do_full[g % DSTAGES], (g / DSTAGES) & 1, abort_flag, p.err);
-        if (ok) ok = wait_bounded(p_ready, g & 1, abort_flag, p.err);
-        if (ok && s == 0 && it > 0) ok = wait_bounded(dkv_empty, (it - 1) & 1, abort_flag, p.err);
+        // ---- A: dV += P^T dO
+        if (!pre_a) ok = ready_a(g, it, s, true);
         if (!ok) break;
         tc_fence_after();
+        const bool pre_b = g == 0 || mbar_test_wait(dq_free, (g - 1) & 1);
+        {
+          const uint64_t db = sdesc_sw128(sdo, BOX, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk)
-          mma_ts(tmem + TM_DV, tmem + TM_S + (kk / 4) * 64 + (kk % 4) * 8, sdesc_sw128(sdo + kk * 2048, BOX, 1024),
-                 id_dkv, (s > 0 || kk > 0) ? 1u : 0u);
-        // dP(g) once dQ^T(g-1) has left the shared columns.  Always issued after dV(g):
-        // its completion (dp_full) then also means dV(g) has finished reading dO(g),
+          for (int kk = 0; kk < BQ / 16; ++kk)
+            mma_ts(tmem + TM_DV, tmem + TM_S + (kk / 4) * 64 + (kk % 4) * 8, sdesc_add(db, kk * 2048), id_dkv,
+                   (s > 0 || kk > 0) ? 1u : 0u);
+        }
+        // ---- B: dP(g) once dQ^T(g-1) has left the shared columns.  Always issued after
+        // dV(g): its completion (dp_full) then also means dV(g) has finished reading dO(g),
         // whose slot the dS warps overwrite with dS^T(g).
-        if (g > 0) ok = wait_bounded(dq_free, (g - 1) & 1, abort_flag, p.err);
+        if (!pre_b) ok = wait_bounded(dq_free, (g - 1) & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
+        const bool pre_c = !next || mbar_test_wait(&q_full[(g + 1) % QSTAGES], ((g + 1) / QSTAGES) & 1);
         issue_kq(tmem + TM_DP, sv, sdo, id_kq);
         mma_commit(dp_full);
-        // S(g+1): its columns held P^T(g), read by the dV MMAs above (issued first)
-        if (s + 1 < nsteps) {
-          ok = wait_bounded(&q_full[(g + 1) % QSTAGES], ((g + 1) / QSTAGES) & 1, abort_flag, p.err);
+        // ---- C: S(g+1): its columns held P^T(g), read by the dV MMAs above (issued first)
+        bool pre_d;
+        if (next) {
+          if (!pre_c) ok = wait_bounded(&q_full[(g + 1) % QSTAGES], ((g + 1) / QSTAGES) & 1, abort_flag, p.err);
           if (!ok) break;
           tc_fence_after();
+          pre_d = mbar_test_wait(ds_ready, g & 1);
           issue_kq(tmem + TM_S, sk, sq0 + ((g + 1) % QSTAGES) * TILE, id_kq);
           mma_commit(s_full);
+        } else {
+          pre_d = mbar_test_wait(ds_ready, g & 1);
         }
-        // dK += dS^T Q ; dQ^T = K^T dS^T (into dP^T's columns, which the dS warps have read)
-        ok = wait_bounded(ds_ready, g & 1, abort_flag, p.err);
+        // ---- D: dQ^T = K^T dS^T (into dP^T's columns, which the dS warps have read), issued
+        // first so that the drain can start early; dK += dS^T Q
+        if (!pre_d) ok = wait_bounded(ds_ready, g & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
+        pre_a = next && ready_a(g + 1, it, s + 1, false);
+        {
+          const uint64_t dds_mn = sdesc_sw128(sdo, BOX, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk)
-          mma_ss(tmem + TM_DK, sdesc_sw128(sdo + (kk / 4) * BOX + (kk % 4) * 32, 16, 1024),
-                 sdesc_sw128(sq + kk * 2048, BOX, 1024), id_dkv, (s > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_ss(tmem + TM_DP, sdesc_sw128(sk + kk * 2048, BOX, 1024), sdesc_add(dds_mn, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+          mma_commit(dq_full);
+          const uint64_t dds_k = sdesc_sw128(sdo, 16, 1024), dq_mn = sdesc_sw128(sq, BOX, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          mma_ss(tmem + TM_DP, sdesc_sw128(sk + kk * 2048, BOX, 1024), sdesc_sw128(sdo + kk * 2048, BOX, 1024),
-                 id_dq, kk > 0 ? 1u : 0u);
-        mma_commit(dq_full);
+          for (int kk = 0; kk < BQ / 16; ++kk)
+            mma_ss(tmem + TM_DK, sdesc_add(dds_k, (kk / 4) * BOX + (kk % 4) * 32), sdesc_add(dq_mn, kk * 2048), id_dkv,
+                   (s > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit(&q_empty[g % QSTAGES]);   // Q(g) and dS^T(g) (in the dO slot) no longer read
         mma_commit(&do_empty[g % DSTAGES]);
       }
@@ -405,15 +433,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int half = 0; half < 2; ++half) {
           const uint32_t* dr = half == 0 ? dr0 : dr1;
           uint32_t pk[16];
+          // dS = P o (dP - delta): the difference in fp32, the product in bf16x2 (keeps
+          // the fp32 pipe, which slows concurrent MMAs when busy, at a low duty)
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
             const float4 d4 = reinterpret_cast<const float4*>(delta_s)[8 * half + c4];
-            const float2 p01 = unpack_bf16x2(pp[16 * half + 2 * c4]);
-            const float2 p23 = unpack_bf16x2(pp[16 * half + 2 * c4 + 1]);
-            pk[2 * c4] = pack_bf16x2(p01.x * (__uint_as_float(dr[4 * c4]) - d4.x),
-                                     p01.y * (__uint_as_float(dr[4 * c4 + 1]) - d4.y));
-            pk[2 * c4 + 1] = pack_bf16x2(p23.x * (__uint_as_float(dr[4 * c4 + 2]) - d4.z),
-                                         p23.y * (__uint_as_float(dr[4 * c4 + 3]) - d4.w));
+            pk[2 * c4] = mul_bf16x2(pp[16 * half + 2 * c4], pack_bf16x2(__uint_as_float(dr[4 * c4]) - d4.x,
+                                                                      __uint_as_float(dr[4 * c4 + 1]) - d4.y));
+            pk[2 * c4 + 1] = mul_bf16x2(pp[16 * half + 2 * c4 + 1],
+                                        pack_bf16x2(__uint_as_float(dr[4 * c4 + 2]) - d4.z,
+                                                    __uint_as_float(dr[4 * c4 + 3]) - d4.w));
           }
 #pragma unroll
           for (int c = 0; c < 4; ++c)
