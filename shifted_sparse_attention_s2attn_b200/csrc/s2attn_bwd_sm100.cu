@@ -40,6 +40,7 @@
 //                   fp32 reduction per (query, warp) into the global accumulator
 //   warp  12        TMA producer (K, V per item; Q + lse and dO + delta through rings)
 //   warp  13        MMA issuer
+//   warp  14        lse converter (-lse * log2(e) in place, once per tile)
 #include "s2_internal.h"
 #include "s2_ptx.cuh"
 
@@ -61,11 +62,11 @@ constexpr uint32_t OFF_DO = OFF_Q + QSTAGES * TILE;    // [DSTAGES] tiles (dO, t
 constexpr uint32_t OFF_LSE = OFF_DO + DSTAGES * TILE;  // [QSTAGES] x lse[128] fp32
 constexpr uint32_t OFF_DELTA = OFF_LSE + QSTAGES * BQ * 4;  // [DSTAGES] x delta[128] fp32
 constexpr uint32_t OFF_BAR = OFF_DELTA + DSTAGES * BQ * 4;
-constexpr int NBARS = 21;
+constexpr int NBARS = 24;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;  // the dynamic smem base must be 1024-byte aligned
 constexpr int NTHREADS = 512;  // warpgroups: P/dS, P/dS, dQ drain, producer + MMA (+2 idle warps)
-constexpr int WARP_DQ0 = 8, WARP_LOAD = 12, WARP_MMA = 13;
+constexpr int WARP_DQ0 = 8, WARP_LOAD = 12, WARP_MMA = 13, WARP_CVT = 14;
 // Launch: 512 threads x 128 registers = 65536.  After setmaxnreg: P/dS warpgroups keep 128,
 // the dQ drain gets 168 (it holds a whole 128-column dQ^T row), producer/MMA drop to 88:
 // 2 x 128 x 128 + 128 x 168 + 128 x 88 = 65536.
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* mma_done = bars + 18;
   uint64_t* dkv_empty = bars + 19;
   uint64_t* drain = bars + 20;
+  uint64_t* lse_ready = bars + 21;  // [3] lse(g) of Q slot g%3 rewritten as -lse*log2(e)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -187,6 +189,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(mma_done, 1);
     mbar_init(dkv_empty, PDS_WARPS);
     mbar_init(drain, 1);
+    for (int s = 0; s < QSTAGES; ++s) mbar_init(&lse_ready[s], 1);
     *abort_flag = (*(volatile int*)p.err != 0) ? 1 : 0;
     fence_mbar_init();
   }
@@ -365,6 +368,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     mma_commit(drain);
     if (!wait_drain(drain, 0)) report_error(p.err, (K_BWD << 8) | SITE_DRAIN);
+   } else if (!skip && warp == WARP_CVT) {
+    // ---------------- lse converter ----------------
+    // Rewrites each tile's lse (natural log, as loaded) in place as -lse * log2(e), so that
+    // the P warps form exp2(s * scale * log2(e) - lse * log2(e)) with one FFMA per element
+    // instead of recomputing the 128 products in each of 256 threads.
+    bool ok = true;
+    int g = 0;
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int nsteps = steps_of(kts[it]);
+      for (int s = 0; s < nsteps; ++s, ++g) {
+        ok = wait_bounded(&q_full[g % QSTAGES], (g / QSTAGES) & 1, abort_flag, p.err);
+        if (!ok) break;
+        float4* l4 = reinterpret_cast<float4*>(smem + OFF_LSE + (g % QSTAGES) * BQ * 4) + lane;
+        float4 v = *l4;
+        v.x *= -LOG2E;
+        v.y *= -LOG2E;
+        v.z *= -LOG2E;
+        v.w *= -LOG2E;
+        *l4 = v;
+        fence_proxy_async_smem();  // the slot is refilled by TMA once the tile is done
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&lse_ready[g % QSTAGES]);
+      }
+    }
+    if (!ok) {
+      report_error(p.err, (K_BWD << 8) | SITE_LOAD);
+      *abort_flag = 1;
+    }
    }
   } else if (wg < 2) {
    if (!skip) {
@@ -381,7 +412,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int s = 0; s < nsteps; ++s, ++g) {
         const float* lse_s = reinterpret_cast<const float*>(smem + OFF_LSE + (g % QSTAGES) * BQ * 4) + 64 * hf;
         const float* delta_s = reinterpret_cast<const float*>(smem + OFF_DELTA + (g % DSTAGES) * BQ * 4) + 64 * hf;
-        ok = wait_bounded(&q_full[g % QSTAGES], (g / QSTAGES) & 1, abort_flag, p.err);
+        ok = wait_bounded(&lse_ready[g % QSTAGES], (g / QSTAGES) & 1, abort_flag, p.err);
         if (ok) ok = wait_bounded(s_full, g & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
@@ -394,8 +425,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const int lim = (s == 0) ? kr - 64 * hf : -1;
 #pragma unroll
           for (int c4 = 0; c4 < 16; ++c4) {
-            const float4 l4 = reinterpret_cast<const float4*>(lse_s)[c4];
-            const float nl[4] = {-l4.x * LOG2E, -l4.y * LOG2E, -l4.z * LOG2E, -l4.w * LOG2E};
+            const float4 l4 = reinterpret_cast<const float4*>(lse_s)[c4];  // -lse * log2(e)
+            const float nl[4] = {l4.x, l4.y, l4.z, l4.w};
             float pv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
