@@ -96,44 +96,42 @@ __device__ __forceinline__ void issue_pv(uint32_t d, uint32_t tp, uint32_t sv, u
 
 // P = exp2(s * sl2 - m) for one 128-column row of S, packed to bf16 pairs and written
 // over the first 64 TMEM columns of S.  Columns c > lim are masked (diagonal tile).
-// Returns the row sum of the fp32 P values (8 partial sums, no long dependency chain).
+// Returns the row sum of the fp32 P values (eight independent partial sums).  The
+// scale-and-shift uses the packed fp32x2 FMA (two elements per instruction): one softmax
+// warp per SM sub-partition is active at a time, so the row is issue-bound around its
+// 128 MUFU exponentials.
 template <bool MASK>
 __device__ __forceinline__ float softmax_p_row(const uint32_t (&s0)[64], const uint32_t (&s1)[64], int lim,
                                                float sl2, float neg_m, uint32_t t_s) {
-  float sp[8];
+  const float2 scale2 = make_float2(sl2, sl2), shift2 = make_float2(neg_m, neg_m);
+  float2 sp[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) sp[e] = 0.f;
-  {
+  for (int e = 0; e < 4; ++e) sp[e] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t(&sr)[64] = h == 0 ? s0 : s1;
     uint32_t pk[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
-      float p0 = ex2_approx(fmaf(__uint_as_float(s0[2 * c]), sl2, neg_m));
-      float p1 = ex2_approx(fmaf(__uint_as_float(s0[2 * c + 1]), sl2, neg_m));
+      const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, shift2);
+      float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
       if (MASK) {
-        p0 = 2 * c <= lim ? p0 : 0.f;
-        p1 = 2 * c + 1 <= lim ? p1 : 0.f;
+        p0 = 64 * h + 2 * c <= lim ? p0 : 0.f;
+        p1 = 64 * h + 2 * c + 1 <= lim ? p1 : 0.f;
       }
-      sp[c % 8] += p0 + p1;
+      sp[c % 4].x += p0; sp[c % 4].y += p1;
       pk[c] = pack_bf16x2(p0, p1);
     }
-    tmem_st_x32(t_s, pk);
+    tmem_st_x32(t_s + 32 * h, pk);
   }
-  {
-    uint32_t pk[32];
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      float p0 = ex2_approx(fmaf(__uint_as_float(s1[2 * c]), sl2, neg_m));
-      float p1 = ex2_approx(fmaf(__uint_as_float(s1[2 * c + 1]), sl2, neg_m));
-      if (MASK) {
-        p0 = 2 * c + 64 <= lim ? p0 : 0.f;
-        p1 = 2 * c + 65 <= lim ? p1 : 0.f;
-      }
-      sp[c % 8] += p0 + p1;
-      pk[c] = pack_bf16x2(p0, p1);
-    }
-    tmem_st_x32(t_s + 32, pk);
-  }
-  return ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+  return ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -341,22 +339,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_ld_x64(t_s + 64, s1);
         // diagonal tile: key column c is visible to row `row` iff c <= row
         const int lim = (t == qt) ? row : 127;
-        // row max: 8 independent partial maxima (a single chain would serialise 128 FMNMX)
+        // row max: 8 independent partial maxima of three-input maxima (a single chain would
+        // serialise the compares)
         float mxp[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
         if (t == qt) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            mxp[c % 8] = fmaxf(mxp[c % 8], c <= lim ? __uint_as_float(s0[c]) : -INFINITY);
-            mxp[c % 8] = fmaxf(mxp[c % 8], c + 64 <= lim ? __uint_as_float(s1[c]) : -INFINITY);
-          }
+          for (int c = 0; c < 64; ++c)
+            mxp[c % 8] = fmax3(mxp[c % 8], c <= lim ? __uint_as_float(s0[c]) : -INFINITY,
+                               c + 64 <= lim ? __uint_as_float(s1[c]) : -INFINITY);
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            mxp[c % 8] = fmaxf(mxp[c % 8], __uint_as_float(s0[c]));
-            mxp[c % 8] = fmaxf(mxp[c % 8], __uint_as_float(s1[c]));
-          }
+          for (int c = 0; c < 64; ++c) mxp[c % 8] = fmax3(mxp[c % 8], __uint_as_float(s0[c]), __uint_as_float(s1[c]));
         }
         const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
                                fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
