@@ -251,31 +251,40 @@ def run_ours(args, w):
         return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
 
     host = {n: make_tensor(w, n) for n in ("q", "k", "v", "dout")}
-    q, k, v, do = (to_dev(host[n]) for n in ("q", "k", "v", "dout"))
-    o = torch.empty_like(q)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    ws_bytes = s2.s2attn_bwd_workspace_bytes(B, N, H, D)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    dq_acc = ws[: B * N * H * D * 4].view(torch.float32)
-    delta_off = ((B * N * H * D * 4 + 255) // 256) * 256
-    delta = ws[delta_off: delta_off + B * H * N * 4].view(torch.float32)
+
+    def buffer_set(inputs=None):
+        """Device tensors of one step: inputs (q, k, v, dout), outputs (o, dq, dk, dv), lse and
+        the backward workspace (fp32 dQ accumulator, delta)."""
+        bs = dict(inputs) if inputs else {n: torch.empty((B, N, H, D), dtype=torch.bfloat16, device=dev)
+                                          for n in ("q", "k", "v", "dout")}
+        for n in ("o", "dq", "dk", "dv"):
+            bs[n] = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=dev)
+        bs["lse"] = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        ws = torch.empty(s2.s2attn_bwd_workspace_bytes(B, N, H, D), dtype=torch.uint8, device=dev)
+        bs["dq_acc"] = ws[: B * N * H * D * 4].view(torch.float32)
+        delta_off = ((B * N * H * D * 4 + 255) // 256) * 256
+        bs["delta"] = ws[delta_off: delta_off + B * H * N * 4].view(torch.float32)
+        return bs
+
+    main_set = buffer_set({n: to_dev(host[n]) for n in ("q", "k", "v", "dout")})
+    q, k, v = main_set["q"], main_set["k"], main_set["v"]
     stream = torch.cuda.current_stream(dev)
 
-    def step(ev=None):
-        s2.rope_pi_apply(q, k, w.pos_scale, w.base, stream)
+    def step(ev=None, bs=main_set, st=stream):
+        s2.rope_pi_apply(bs["q"], bs["k"], w.pos_scale, w.base, st)
         if ev is not None:
-            ev[0].record(stream)
-        s2.s2attn_fwd(q, k, v, o, lse, G, SH, stream)
+            ev[0].record(st)
+        s2.s2attn_fwd(bs["q"], bs["k"], bs["v"], bs["o"], bs["lse"], G, SH, st)
         if ev is not None:
-            ev[1].record(stream)
-        s2.s2attn_bwd_preprocess(o, do, delta, dq_acc, stream)
+            ev[1].record(st)
+        s2.s2attn_bwd_preprocess(bs["o"], bs["dout"], bs["delta"], bs["dq_acc"], st)
         if ev is not None:
-            ev[2].record(stream)
-        s2.s2attn_bwd_main(q, k, v, do, lse, delta, dq_acc, dk, dv, G, SH, stream)
+            ev[2].record(st)
+        s2.s2attn_bwd_main(bs["q"], bs["k"], bs["v"], bs["dout"], bs["lse"], bs["delta"], bs["dq_acc"], bs["dk"],
+                           bs["dv"], G, SH, st)
         if ev is not None:
-            ev[3].record(stream)
-        s2.s2attn_bwd_dq_convert(dq_acc, dq, stream)
+            ev[3].record(st)
+        s2.s2attn_bwd_dq_convert(bs["dq_acc"], bs["dq"], st)
 
     def barrier():
         if world > 1:
@@ -310,33 +319,81 @@ def run_ours(args, w):
 
     ms_max = max_over_ranks(ms, dev)
 
+    # ---- full causal attention (inference case: one group, no shift), forward only ----
+    pairs_full = B * H * N * (N + 1) // 2
+    fc_lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    fc_o = torch.empty_like(q)
+    for _ in range(2):
+        s2.s2attn_fwd(q, k, v, fc_o, fc_lse, N, 0, stream)
+    fc0, fc1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fc_reps = 5
+    fc0.record(stream)
+    for _ in range(fc_reps):
+        s2.s2attn_fwd(q, k, v, fc_o, fc_lse, N, 0, stream)
+    fc1.record(stream)
+    torch.cuda.synchronize(dev)
+    fc_ms = fc0.elapsed_time(fc1) / fc_reps
+    del fc_o, fc_lse
+
     # ---- end to end: host buffers in, results out, through the same public calls ----
+    # Each step copies its inputs from pinned host memory and its results back.  Steps are
+    # pipelined over three streams with two device buffer sets: the host->device copy of
+    # step i+1 and the device->host copy of step i-1 overlap the compute of step i.
     e2e_steps = max(3, min(args.steps, 10))
     pinned = {n: torch.from_numpy(host[n].view(np.int16)).view(torch.bfloat16).pin_memory() for n in host}
-    outs = {n: torch.empty((B, N, H, D), dtype=torch.bfloat16).pin_memory() for n in ("o", "dq", "dk", "dv")}
-    dev_in = {"q": q, "k": k, "v": v, "dout": do}
-    dev_out = {"o": o, "dq": dq, "dk": dk, "dv": dv}
+    sets = [main_set, buffer_set()]
+    outs = [{n: torch.empty((B, N, H, D), dtype=torch.bfloat16).pin_memory() for n in ("o", "dq", "dk", "dv")}
+            for _ in sets]
     h2d = sum(x.numel() * x.element_size() for x in pinned.values())
-    d2h = sum(x.numel() * x.element_size() for x in outs.values())
+    d2h = sum(x.numel() * x.element_size() for x in outs[0].values())
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        for n in pinned:
-            dev_in[n].copy_(pinned[n], non_blocking=True)
-        step()
-        for n in outs:
-            outs[n].copy_(dev_out[n], non_blocking=True)
+    def e2e_run(nsteps, e_start=None, e_end=None):
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        h2d_done, cmp_done, d2h_done = [None, None], [None, None], [None, None]
+        if e_start is not None:
+            e_start.record(stream)
+            s_h2d.wait_event(e_start)
+            s_d2h.wait_event(e_start)
+        for i in range(nsteps):
+            slot = i % 2
+            bs = sets[slot]
+            with torch.cuda.stream(s_h2d):  # inputs of step i, once step i-2 stopped reading them
+                if cmp_done[slot] is not None:
+                    s_h2d.wait_event(cmp_done[slot])
+                for n in pinned:
+                    bs[n].copy_(pinned[n], non_blocking=True)
+                h2d_done[slot] = ev()
+                h2d_done[slot].record(s_h2d)
+            stream.wait_event(h2d_done[slot])
+            if d2h_done[slot] is not None:  # outputs of step i-2 copied out
+                stream.wait_event(d2h_done[slot])
+            step(bs=bs, st=stream)
+            cmp_done[slot] = ev()
+            cmp_done[slot].record(stream)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(cmp_done[slot])
+                for n in outs[slot]:
+                    outs[slot][n].copy_(bs[n], non_blocking=True)
+                d2h_done[slot] = ev()
+                d2h_done[slot].record(s_d2h)
+        if e_end is not None:
+            for e in h2d_done + d2h_done:
+                if e is not None:
+                    stream.wait_event(e)
+            e_end.record(stream)
 
-    e2e_step()
+    e2e_run(2)
     torch.cuda.synchronize(dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e2e_run(e2e_steps, e0, e1)
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    rc, detail = s2.get_device_error()
+    if rc != 0:
+        raise SystemExit(f"device error word set during the end-to-end run: {detail:#x}")
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -368,7 +425,10 @@ def run_ours(args, w):
                          "frac": fwd_flops / fwd_avg / 1e12 / peak_sus,
                          "traffic": traffic_record("s2attn_fwd_sm100.cu", "s2attn_fwd_kernel")},
         "e2e": {"value": whole_job_tflops(flops, e2e_steps, world, e2e_ms), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "overlap": "H2D of step i+1 and D2H of step i-1 run on their own streams during step i"},
+        "full_causal_fwd": {"workload": f"{w.name} with G=N={N}, shift_heads=0 (inference: full causal attention)",
+                            "ms": fc_ms, "tflops": 4 * D * pairs_full / (fc_ms / 1e3) / 1e12},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks,
     }
