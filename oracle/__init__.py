@@ -8,7 +8,9 @@ file only marshals numpy arrays into it.
 Pinned by tests/test_oracle_pins.py against: textbook causal attention (torch
 SDPA in fp64) for G=N without shift; brute force with an explicit N x N mask for
 grouped and shifted heads; the shift example of the "LongLoRA paper notes" page
-(section 3.3); central finite differences for the gradients; RoPE invariants.
+(section 3.3); central finite differences for the gradients; RoPE invariants; for the
+decoding step, torch SDPA with an explicit mask, the last rows of full causal
+attention, and closed forms.
 """
 import ctypes
 import numpy as np
@@ -33,6 +35,8 @@ def _load():
         lib.oracle_s2attn_fwd_full.restype = i
         lib.oracle_s2attn_bwd_full.argtypes = [i, vp, vp, vp, vp, i, i, i, i, i, i, dp, dp, dp]
         lib.oracle_s2attn_bwd_full.restype = i
+        lib.oracle_decode.argtypes = [i, vp, vp, vp, i, i, i, i, i, dp, dp]
+        lib.oracle_decode.restype = i
         lib.oracle_rope_pi_f64.argtypes = [vp, vp, i, i, i, i, ctypes.c_double, ctypes.c_double]
         lib.oracle_rope_pi_f64.restype = None
         lib.oracle_rope_pi_f32_bf16.argtypes = [vp, vp, i, i, i, i, ctypes.c_float, ctypes.c_float]
@@ -114,6 +118,23 @@ def s2attn_unit(q, k, v, G, shift_heads, b, h, j, qrows=(), krows=(), dout=None)
     if nk:
         out.update(dk=dk[:nk], dv=dv[:nk], ktok=ktok[:nk])
     return out
+
+
+def decode(q, k, v):
+    """Full causal attention of the last M positions (a decoding step).
+
+    q: [B,M,H,D], query m at position N-M+m; k, v: [B,N,H,D] (all N positions).
+    Returns (o [B,M,H,D] f64, lse [B,H,M] f64)."""
+    (q, k, v), code = _prep(q, k, v)
+    B, M, H, D = q.shape
+    N = k.shape[1]
+    if k.shape != (B, N, H, D) or v.shape != k.shape:
+        raise ValueError("oracle: k and v must be [B,N,H,D] with q's B, H, D")
+    o = np.empty((B, M, H, D), np.float64)
+    lse = np.empty((B, H, M), np.float64)
+    if _load().oracle_decode(code, _ptr(q), _ptr(k), _ptr(v), B, M, N, H, D, _ptr(o), _ptr(lse)):
+        raise ValueError("oracle: invalid decode sizes")
+    return o, lse
 
 
 def rope_pi_f64(x, pos_scale, base=10000.0):

@@ -299,6 +299,53 @@ int oracle_s2attn_bwd_full(int dtype, const void *q, const void *k, const void *
   return rc;
 }
 
+/* ---- decoding: full causal attention for the last M positions ------------- */
+
+/*
+ * Inference runs ordinary full attention, not S^2-Attn ("LongLoRA paper notes",
+ * section 3.1; model.aibase.cn, features list).  A decoding step appends M new
+ * tokens to a sequence of N positions: k, v [B,N,H,D] hold all N positions
+ * (the new ones included), q [B,M,H,D] holds the M new queries, query m sits at
+ * position N - M + m and sees the keys at positions 0 .. N - M + m.
+ * Writes o [B,M,H,D] and lse [B,H,M] (natural log of sum_t exp(scale*q.k_t)).
+ * Returns 0, or -1 on bad sizes (M < 1, M > N, ...).
+ */
+int oracle_decode(int dtype, const void *q, const void *k, const void *v,
+                  int B, int M, int N, int H, int D, double *o, double *lse) {
+  if (B < 1 || M < 1 || N < 1 || H < 1 || D < 1 || M > N) return -1;
+  const double scale = 1.0 / sqrt((double)D);
+#pragma omp parallel
+  {
+    double *qrow = malloc(sizeof(double) * (size_t)D);
+    double *krow = malloc(sizeof(double) * (size_t)D);
+    double *S = malloc(sizeof(double) * (size_t)N);
+#pragma omp for collapse(3) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b)
+      for (int h = 0; h < H; ++h)
+        for (int m = 0; m < M; ++m) {
+          const long pos = (long)N - M + m; /* last visible key */
+          for (int d = 0; d < D; ++d) qrow[d] = widen(q, idx_bnhd(b, m, h, d, M, H, D), dtype);
+          double mx = -INFINITY;
+          for (long t = 0; t <= pos; ++t) {
+            for (int d = 0; d < D; ++d) krow[d] = widen(k, idx_bnhd(b, t, h, d, N, H, D), dtype);
+            S[t] = scale * dot(qrow, krow, D);
+            if (S[t] > mx) mx = S[t];
+          }
+          double l = 0.0;
+          for (long t = 0; t <= pos; ++t) l += exp(S[t] - mx);
+          double *orow = o + idx_bnhd(b, m, h, 0, M, H, D);
+          for (int d = 0; d < D; ++d) orow[d] = 0.0;
+          for (long t = 0; t <= pos; ++t) {
+            double p = exp(S[t] - mx) / l;
+            for (int d = 0; d < D; ++d) orow[d] += p * widen(v, idx_bnhd(b, t, h, d, N, H, D), dtype);
+          }
+          lse[((size_t)b * H + h) * M + m] = mx + log(l);
+        }
+    free(qrow); free(krow); free(S);
+  }
+  return 0;
+}
+
 /* ---- RoPE with position interpolation ------------------------------------ */
 
 /* fp64 reference.  Token t sits at interpolated position t * pos_scale; pair
