@@ -335,6 +335,30 @@ def run_ours(args, w):
     fc_ms = fc0.elapsed_time(fc1) / fc_reps
     del fc_o, fc_lse
 
+    # ---- decoding step (inference, full causal attention of the last M positions) ----
+    # The queries are the last M rows of q; K and V (0.54 GB, larger than L2) are read
+    # once per call, which makes the step HBM-bound.
+    decode = {}
+    for M in (1, 16):
+        dq_ = q[:, N - M:].contiguous()
+        d_o = torch.empty_like(dq_)
+        d_lse = torch.empty((B, H, M), dtype=torch.float32, device=dev)
+        d_ws = torch.empty(s2.s2attn_decode_workspace_bytes(B, M, N, H, D), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            s2.s2attn_decode(dq_, k, v, d_o, d_lse, d_ws, stream)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d_reps = 20
+        d0.record(stream)
+        for _ in range(d_reps):
+            s2.s2attn_decode(dq_, k, v, d_o, d_lse, d_ws, stream)
+        d1.record(stream)
+        torch.cuda.synchronize(dev)
+        d_ms = d0.elapsed_time(d1) / d_reps
+        kv_bytes = 2 * B * N * H * D * 2
+        decode[f"M{M}"] = {"ms": d_ms, "kv_bytes": kv_bytes, "gbs": kv_bytes / (d_ms / 1e3) / 1e9,
+                           "tokens_per_s": B * M / (d_ms / 1e3)}
+        del dq_, d_o, d_lse, d_ws
+
     # ---- end to end: host buffers in, results out, through the same public calls ----
     # Each step copies its inputs from pinned host memory and its results back.  Steps are
     # pipelined over three streams with two device buffer sets: the host->device copy of
@@ -429,6 +453,11 @@ def run_ours(args, w):
                 "overlap": "H2D of step i+1 and D2H of step i-1 run on their own streams during step i"},
         "full_causal_fwd": {"workload": f"{w.name} with G=N={N}, shift_heads=0 (inference: full causal attention)",
                             "ms": fc_ms, "tflops": 4 * D * pairs_full / (fc_ms / 1e3) / 1e12},
+        "decode": {"workload": f"{w.name}: the last M rows of q as decoding queries (query m at position "
+                               f"N-M+m) against all N={N} positions of k, v; full causal attention",
+                   "bound": "hbm", "peak_gbs": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
+                   **{k_: dict(v_, frac=v_["gbs"] / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+                      for k_, v_ in decode.items()}},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks,
     }

@@ -100,6 +100,26 @@ int s2attn_bwd_main(const void* q, const void* k, const void* v, const void* dou
 int s2attn_bwd_dq_convert(const float* dq_acc, void* dq, int B, int N, int H, int D, void* stream);
 
 /*
+ * Decoding step of full causal attention (inference).  Inference runs ordinary
+ * full attention, not S^2-Attn ("LongLoRA paper notes", section 3.1; model.aibase.cn,
+ * features list: the shifted attention is only needed in training).  A step appends
+ * M new tokens to a sequence of N positions:
+ *   q    : [B,M,H,D] bf16, the new queries; query m sits at position N-M+m
+ *   k, v : [B,N,H,D] bf16, all N positions (the M new ones included)
+ *   o    : [B,M,H,D] bf16 output; query m attends to the keys at positions
+ *          0 .. N-M+m with scale 1/sqrt(D)
+ *   lse  : [B,H,M] fp32 output, natural log of sum over those keys of exp(scale*q.k)
+ * Requirements: 1 <= M <= N; M <= 16 and D == 128 (else S2ATTN_ERR_UNSUPPORTED).
+ * `workspace` (device, caller-owned, 256-byte aligned, at least
+ * s2attn_decode_workspace_bytes bytes) receives per-split partial results and is
+ * overwritten.  V rows past a query's causal limit are multiplied by a zero weight,
+ * so k and v must hold finite values at every position.  Runs two kernels on `stream`.
+ */
+size_t s2attn_decode_workspace_bytes(int B, int M, int N, int H, int D);
+int s2attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int M, int N, int H,
+                  int D, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fp32 forward/backward on CUDA cores, any valid shape with 1 <= D <= 128
  * (G >= 1 divides N; G even when shift_heads > 0).  Same tensor layouts, all fp32.
  * s2attn_bwd_f32 uses the delta part of the workspace only
@@ -154,7 +174,7 @@ int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* 
 /*
  * Reads the current device's error word: S2ATTN_OK if no kernel has failed since
  * the last clear, else S2ATTN_ERR_DEVICE_TIMEOUT with *detail (if non-NULL) set to
- * (kernel << 8) | site (kernel 1 = forward, 2 = backward).  Synchronize the streams
+ * (kernel << 8) | site (kernel 1 = forward, 2 = backward, 4 = decoding step).  Synchronize the streams
  * that ran library kernels first.
  */
 int s2attn_get_device_error(int* detail);

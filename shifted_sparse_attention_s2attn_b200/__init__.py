@@ -12,7 +12,7 @@ import os
 __all__ = [
     "S2AttnError", "capi", "library_path",
     "s2attn_fwd", "s2attn_bwd", "s2attn_bwd_workspace_bytes", "s2attn_bwd_preprocess", "s2attn_bwd_main",
-    "s2attn_bwd_dq_convert", "s2attn_bwd_noalloc", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply",
+    "s2attn_bwd_dq_convert", "s2attn_bwd_noalloc", "s2attn_decode", "s2attn_decode_workspace_bytes", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply",
     "get_device_error", "clear_device_error", "s2attn_selftest_bounded_wait",
 ]
 
@@ -52,6 +52,8 @@ def capi():
         "s2attn_bwd_main": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P], I),
         "s2attn_bwd_dq_convert": ([P, P, I, I, I, I, P], I),
         "s2attn_bwd_noalloc": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P], I),
+        "s2attn_decode_workspace_bytes": ([I, I, I, I, I], Z),
+        "s2attn_decode": ([P, P, P, P, P, I, I, I, I, I, P, Z, P], I),
         "s2attn_fwd_f32": ([P, P, P, P, P, I, I, I, I, I, I, P], I),
         "s2attn_bwd_f32": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, Z, P], I),
         "rope_pi_apply": ([P, P, I, I, I, I, F, F, P], I),
@@ -138,6 +140,21 @@ def s2attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, stream
     _check("s2attn_bwd_noalloc", capi().s2attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout),
                                                            _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, D, G,
                                                            shift_heads, _stream(stream)))
+
+
+def s2attn_decode_workspace_bytes(B, M, N, H, D):
+    return int(capi().s2attn_decode_workspace_bytes(B, M, N, H, D))
+
+
+def s2attn_decode(q, k, v, o, lse, workspace, stream=None):
+    """Decoding step of full causal attention: q [B,M,H,D] (query m at position N-M+m)
+    against k, v [B,N,H,D]; o [B,M,H,D] bf16 and lse [B,H,M] fp32 are written.
+    workspace: a uint8 device tensor of at least s2attn_decode_workspace_bytes bytes."""
+    B, M, H, D = _bnhd(q, "q")
+    N = _bnhd(k, "k")[1]
+    _check("s2attn_decode", capi().s2attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, M, N, H, D,
+                                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                 _stream(stream)))
 
 
 def s2attn_fwd_f32(q, k, v, o, lse, G, shift_heads, stream=None):

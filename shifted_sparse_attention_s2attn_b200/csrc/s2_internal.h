@@ -10,7 +10,7 @@ namespace s2 {
 
 // Device error codes (first failure wins; read with s2attn_get_device_error).
 // code = (kernel << 8) | site
-enum Kernel : int { K_FWD = 1, K_BWD = 2, K_SELFTEST = 3 };
+enum Kernel : int { K_FWD = 1, K_BWD = 2, K_SELFTEST = 3, K_DEC = 4 };
 
 // Problem description after validation.  Rows of a [B,N,H,D] tensor for head h
 // are addressed through 3-D tensor maps with dims {D, H, B*N}.
@@ -40,6 +40,18 @@ cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float
 cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* dout,
                            const float* lse, float* dq, float* dk, float* dv, float* delta, const Shape& s,
                            cudaStream_t st);
+
+// Decoding step (full causal attention of the last M <= 16 positions), D == 128.
+// The K/V of each (b, h) is cut into `S` splits of `tiles_per_split` 128-key tiles
+// (decode_splits picks them for `n_sm` SMs, at most kDecodeMaxSplits); the split kernel
+// writes fp32 partials (part_o [B*H][S][M][128], part_ml [B*H][S][M][2]) and a second
+// kernel combines them into o and lse.  Tensor maps: 128-row boxes of 64 columns,
+// 128-byte swizzle, over k and v ([B,N,H,D]).
+constexpr int kDecodeMaxSplits = 64;
+int decode_splits(int B, int N, int H, int n_sm, int* tiles_per_split);
+cudaError_t launch_decode_sm100(const CUtensorMap& tk, const CUtensorMap& tv, const void* q, void* o, float* lse,
+                                float* part_o, float* part_ml, int B, int M, int N, int H, int S,
+                                int tiles_per_split, int* err, cudaStream_t st);
 
 // RoPE-PI in place on bf16 q and k, with a cos/sin table [N, D/2] (fp32 each).
 cudaError_t launch_rope_pi(void* q, void* k, const float* cos_tab, const float* sin_tab, int B, int N, int H,

@@ -174,6 +174,41 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout,
   return cuda_status(s2::launch_bwd_sm100(tq, tk, tv, tdo, lse, delta, dq_acc, dk, dv, s, err, st));
 }
 
+// SM count of the current device, looked up once per device.
+int sm_count() {
+  static std::mutex mu;
+  static int cache[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev] && cudaDeviceGetAttribute(&cache[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    cache[dev] = 0;
+  return cache[dev];
+}
+
+constexpr int kDecodeMaxM = 16;
+
+int check_decode_shape(int B, int M, int N, int H, int D) {
+  if (B < 1 || M < 1 || N < 1 || H < 1 || D < 1 || M > N) return S2ATTN_ERR_INVALID_ARG;
+  if ((long long)B * N > INT_MAX / 2) return S2ATTN_ERR_INVALID_ARG;
+  if ((long long)B * N * H > (LLONG_MAX / 8) / D) return S2ATTN_ERR_INVALID_ARG;
+  if (D != 128 || M > kDecodeMaxM) return S2ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * H * M > INT_MAX || (long long)B * H * s2::kDecodeMaxSplits > INT_MAX)
+    return S2ATTN_ERR_UNSUPPORTED;
+  return S2ATTN_OK;
+}
+
+// Splits the workspace is sized for: the most any device can get (1 per 128-key tile,
+// at most kDecodeMaxSplits), so that the size does not depend on the device.
+int decode_max_splits(int N) {
+  const int tiles = (N + 127) / 128;
+  return tiles < s2::kDecodeMaxSplits ? tiles : s2::kDecodeMaxSplits;
+}
+
+size_t decode_part_o_bytes(int B, int M, int N, int H, int D) {
+  return align256((size_t)B * H * decode_max_splits(N) * M * D * sizeof(float));
+}
+
 }  // namespace
 
 extern "C" {
@@ -261,6 +296,36 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   if ((rc = cuda_status(s2::launch_bwd_preprocess(o, dout, delta, dq_acc, s, st)))) return rc;
   if ((rc = bwd_main_impl(q, k, v, dout, lse, delta, dq_acc, dk, dv, s, st))) return rc;
   return cuda_status(s2::launch_dq_convert(dq_acc, dq, s, st));
+}
+
+size_t s2attn_decode_workspace_bytes(int B, int M, int N, int H, int D) {
+  if (check_decode_shape(B, M, N, H, D)) return 0;
+  return decode_part_o_bytes(B, M, N, H, D) +
+         align256((size_t)B * H * decode_max_splits(N) * M * 2 * sizeof(float));
+}
+
+int s2attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int M, int N, int H,
+                  int D, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_decode_shape(B, M, N, H, D);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return S2ATTN_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < s2attn_decode_workspace_bytes(B, M, N, H, D) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return S2ATTN_ERR_WORKSPACE;
+  const int n_sm = sm_count();
+  if (n_sm <= 0) return S2ATTN_ERR_CUDA;
+  int tps = 0;
+  const int S = s2::decode_splits(B, N, H, n_sm, &tps);
+  float* part_o = static_cast<float*>(workspace);
+  float* part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_part_o_bytes(B, M, N, H, D));
+  const s2::Shape s{B, N, H, D, N, 0};
+  CUtensorMap tk, tv;
+  if (!map_bf16_sw128(&tk, k, s, 128) || !map_bf16_sw128(&tv, v, s, 128)) return S2ATTN_ERR_CUDA;
+  int* err = error_word_ptr();
+  if (!err) return S2ATTN_ERR_CUDA;
+  return cuda_status(s2::launch_decode_sm100(tk, tv, q, o, lse, part_o, part_ml, B, M, N, H, S, tps, err,
+                                             static_cast<cudaStream_t>(stream)));
 }
 
 int s2attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int N, int H, int D,

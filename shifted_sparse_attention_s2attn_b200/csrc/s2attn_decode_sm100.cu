@@ -1,0 +1,378 @@
+// s2attn_decode_sm100.cu -- a decoding step of full causal attention on B200 (sm_100a).
+//
+// Inference runs ordinary full attention; S^2-Attn is a training-time device only
+// ("LongLoRA paper notes", section 3.1; model.aibase.cn, features list).  A decoding
+// step appends M (<= 16) tokens to a sequence of N positions: k, v [B,N,H,D] hold all
+// N positions (the new ones included), q [B,M,H,D] the M new queries; query m sits at
+// position N-M+m and sees keys 0 .. N-M+m.
+//
+// With a handful of queries the step is a matrix-vector product over the whole K/V of
+// every head: 2*N*D*2 bytes per head and 4*M*D FLOPs per key, so it is bound by HBM, not
+// by arithmetic -- it runs on the CUDA cores, and its job is to stream K and V at full
+// bandwidth:
+//   * split-KV: CTA (b, h, split) takes a run of 128-key tiles of one head, so that the
+//     grid fills every SM even for one sequence (B*H*splits CTAs);
+//   * a producer thread streams the tiles with TMA (four 128-row x 64-column boxes per
+//     tile: K and V, two column halves each, 128-byte swizzle) through a 3-stage ring;
+//   * 4 consumer warps take 32 keys of each tile: lane = key for Q.K (16-byte swizzled
+//     row reads, conflict-free), an online base-2 softmax per warp, then lane = 4 head
+//     dims for P.V (the probabilities broadcast from shared memory);
+//   * the warps' partial (max, sum, unnormalised output) merge in shared memory and the
+//     CTA writes one fp32 partial per (b, h, split, m); a second kernel combines the
+//     splits into o (bf16) and lse.
+#include "s2_internal.h"
+#include "s2_ptx.cuh"
+
+namespace s2 {
+namespace dec {
+
+constexpr int HD = 128;
+constexpr int TK = 128;                       // keys per tile
+constexpr uint32_t BOX = TK * 128;            // 128 rows x 128 B (64 bf16 columns)
+constexpr uint32_t TILE_BYTES = 4 * BOX;      // K box 0, K box 1, V box 0, V box 1
+constexpr int NST = 3;                        // ring stages
+constexpr int MAXM = 16;
+constexpr int NCW = 4;                        // consumer warps
+constexpr int NTHREADS = (NCW + 1) * 32;      // + producer warp
+constexpr uint32_t OFF_Q = NST * TILE_BYTES;              // float [MAXM][HD], scaled to the log2 domain
+constexpr uint32_t OFF_P = OFF_Q + MAXM * HD * 4;         // float [NCW][32 keys][MT]
+constexpr uint32_t OFF_BAR = OFF_P + NCW * 32 * MAXM * 4;
+constexpr uint32_t OFF_MISC = OFF_BAR + 2 * NST * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;     // + slack to align the base to 1024 B
+constexpr float LOG2E = 1.4426950408889634f;
+
+struct Params {
+  const __nv_bfloat16* q;
+  float* part_o;   // [B*H][S][M][HD] unnormalised
+  float* part_ml;  // [B*H][S][M][2]  (running max in the log2 domain, sum)
+  int B, M, N, H, S, tiles_per_split;
+  float qscale;    // log2(e) / sqrt(D)
+  int* err;
+};
+
+enum Site : int { SITE_LOAD = 1, SITE_CONSUME = 2, SITE_DRAIN = 3 };
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                        const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + NST;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC);
+  float* qs = reinterpret_cast<float*>(smem + OFF_Q);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int split = (int)(blockIdx.x % p.S);
+  const int bh = (int)(blockIdx.x / p.S);
+  const int h = bh % p.H, b = bh / p.H;
+  const int t_begin = split * p.tiles_per_split * TK;
+  const int t_end = min(p.N, t_begin + p.tiles_per_split * TK);
+  const int n_tiles = t_end > t_begin ? (t_end - t_begin + TK - 1) / TK : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NCW);
+    }
+    *abort_flag = (*(volatile int*)p.err != 0) ? 1 : 0;
+    fence_mbar_init();
+  }
+  // queries of this head, scaled into the log2 domain; rows m >= M are zero
+  if (threadIdx.x < HD) {
+    const int d = threadIdx.x;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      float x = 0.0f;
+      if (m < p.M) x = __bfloat162float(p.q[((size_t)(b * p.M + m) * p.H + h) * HD + d]) * p.qscale;
+      qs[m * HD + d] = x;
+    }
+  }
+  __syncthreads();
+  const bool skip = *abort_flag != 0;
+
+  if (warp == NCW) {
+    // ---------------- TMA producer ----------------
+    if (!skip && lane == 0) {
+      prefetch_tmap(&tk);
+      prefetch_tmap(&tv);
+      bool ok = true;
+      int issued = 0;
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int slot = i % NST;
+        if (i >= NST) ok = wait_bounded(&empty[slot], ((i / NST) - 1) & 1, abort_flag, p.err);
+        if (!ok) break;
+        uint8_t* dst = smem + slot * TILE_BYTES;
+        const int row = b * p.N + t_begin + i * TK;
+        mbar_arrive_expect_tx(&full[slot], TILE_BYTES);
+        tma_load_3d(dst, &tk, 0, h, row, &full[slot]);
+        tma_load_3d(dst + BOX, &tk, 64, h, row, &full[slot]);
+        tma_load_3d(dst + 2 * BOX, &tv, 0, h, row, &full[slot]);
+        tma_load_3d(dst + 3 * BOX, &tv, 64, h, row, &full[slot]);
+        issued = i + 1;
+      }
+      if (!ok) {
+        report_error(p.err, (K_DEC << 8) | SITE_LOAD);
+        *abort_flag = 1;
+      }
+      bool dok = true;
+      for (int i = (issued > NST ? issued - NST : 0); i < issued; ++i)
+        dok &= wait_drain(&full[i % NST], (i / NST) & 1);
+      if (!dok) report_error(p.err, (K_DEC << 8) | SITE_DRAIN);
+    }
+    return;  // the producer warp takes no part in the merge below
+  }
+
+  // ---------------- consumers: 32 keys of each tile per warp ----------------
+  float m_run[MT], l_lane[MT], o_acc[MT][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    m_run[m] = -INFINITY;
+    l_lane[m] = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o_acc[m][e] = 0.0f;
+  }
+  const float4* q4 = reinterpret_cast<const float4*>(qs);
+  float* pbuf = reinterpret_cast<float*>(smem + OFF_P) + warp * 32 * MT;
+  const int lim0 = p.N - p.M;  // query m sees keys t <= lim0 + m
+  bool ok = !skip;
+  for (int i = 0; i < n_tiles && ok; ++i) {
+    const int slot = i % NST;
+    ok = wait_bounded(&full[slot], (i / NST) & 1, abort_flag, p.err);
+    if (!ok) break;
+    const uint8_t* kb = smem + slot * TILE_BYTES;
+    const uint8_t* vb = kb + 2 * BOX;
+    const int t0 = t_begin + i * TK + 32 * warp;  // first key of this warp's 32
+    // ---- scores, lane = key: s_m = (q_m * log2e / sqrt(D)) . k_t
+    const int r = 32 * warp + lane;
+    const int t = t0 + lane;
+    float s[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) s[m] = 0.0f;
+#pragma unroll 4
+    for (int c = 0; c < HD / 8; ++c) {
+      const uint4 kw = *reinterpret_cast<const uint4*>(kb + (c >> 3) * BOX + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+      float kf[8];
+      bf16x8_to_f32(kw, kf);
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const float4 qa = q4[(m * HD + 8 * c) / 4], qb = q4[(m * HD + 8 * c) / 4 + 1];
+        float a = s[m];
+        a = fmaf(qa.x, kf[0], a);
+        a = fmaf(qa.y, kf[1], a);
+        a = fmaf(qa.z, kf[2], a);
+        a = fmaf(qa.w, kf[3], a);
+        a = fmaf(qb.x, kf[4], a);
+        a = fmaf(qb.y, kf[5], a);
+        a = fmaf(qb.z, kf[6], a);
+        a = fmaf(qb.w, kf[7], a);
+        s[m] = a;
+      }
+    }
+    // ---- online softmax over this warp's 32 keys (keys past the split or the causal
+    // limit of query m count as -inf)
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const bool vis = t < t_end && t <= lim0 + m;
+      const float sm = vis ? s[m] : -INFINITY;
+      const float m_new = fmaxf(m_run[m], warp_max(sm));
+      float pr = 0.0f;
+      if (m_new != -INFINITY) {  // warp-uniform
+        if (m_new != m_run[m]) {
+          const float alpha = ex2_approx(m_run[m] - m_new);  // 0 while m_run is -inf
+          l_lane[m] *= alpha;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o_acc[m][e] *= alpha;
+          m_run[m] = m_new;
+        }
+        pr = vis ? ex2_approx(sm - m_new) : 0.0f;
+      }
+      l_lane[m] += pr;
+      pbuf[lane * MT + m] = pr;
+    }
+    __syncwarp();
+    // ---- o += p . v, lane = head dims [4*lane, 4*lane + 4)
+    const int nv = min(32, t_end - t0);  // keys of this warp that exist (warp-uniform)
+    const uint32_t vcol = (lane >> 4) * BOX + (lane & 1) * 8;
+    const int vchunk = (lane & 15) >> 1;
+    for (int j = 0; j < nv; ++j) {
+      const int rr = 32 * warp + j;
+      const uint2 vw = *reinterpret_cast<const uint2*>(vb + vcol + rr * 128 + ((vchunk ^ (rr & 7)) << 4));
+      const float v0 = __uint_as_float(vw.x << 16), v1 = __uint_as_float(vw.x & 0xffff0000u);
+      const float v2 = __uint_as_float(vw.y << 16), v3 = __uint_as_float(vw.y & 0xffff0000u);
+      const float* pj = pbuf + j * MT;
+      if constexpr (MT >= 4) {
+#pragma unroll
+        for (int m = 0; m < MT; m += 4) {
+          const float4 p4 = *reinterpret_cast<const float4*>(pj + m);
+          const float pm[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            o_acc[m + u][0] = fmaf(pm[u], v0, o_acc[m + u][0]);
+            o_acc[m + u][1] = fmaf(pm[u], v1, o_acc[m + u][1]);
+            o_acc[m + u][2] = fmaf(pm[u], v2, o_acc[m + u][2]);
+            o_acc[m + u][3] = fmaf(pm[u], v3, o_acc[m + u][3]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float pm = pj[m];
+          o_acc[m][0] = fmaf(pm, v0, o_acc[m][0]);
+          o_acc[m][1] = fmaf(pm, v1, o_acc[m][1]);
+          o_acc[m][2] = fmaf(pm, v2, o_acc[m][2]);
+          o_acc[m][3] = fmaf(pm, v3, o_acc[m][3]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+  }
+  if (!ok && !skip) {
+    report_error(p.err, (K_DEC << 8) | SITE_CONSUME);
+    *abort_flag = 1;
+  }
+
+  // ---------------- merge the 4 warps' partials (consumer threads only) ----------------
+  // Every tile has been consumed, so no copy is in flight and the ring's memory is free.
+  named_bar_sync(1, NCW * 32);
+  float* wo = reinterpret_cast<float*>(smem);                 // [NCW][MT][HD]
+  float* wml = wo + NCW * MT * HD;                            // [NCW][MT][2]
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const float l = warp_sum(l_lane[m]);
+    *reinterpret_cast<float4*>(wo + (warp * MT + m) * HD + 4 * lane) =
+        make_float4(o_acc[m][0], o_acc[m][1], o_acc[m][2], o_acc[m][3]);
+    if (lane == 0) {
+      wml[(warp * MT + m) * 2] = m_run[m];
+      wml[(warp * MT + m) * 2 + 1] = l;
+    }
+  }
+  named_bar_sync(1, NCW * 32);
+  if (skip || *abort_flag) return;
+  const int d = threadIdx.x;  // 0 .. 127
+  const size_t part = (size_t)bh * p.S + split;
+  for (int m = 0; m < p.M; ++m) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, wml[(w * MT + m) * 2]);
+    float l = 0.0f, o = 0.0f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        const float wm = wml[(w * MT + m) * 2];
+        const float wgt = ex2_approx(wm - mx);  // 0 for a warp that saw no visible key
+        l += wgt * wml[(w * MT + m) * 2 + 1];
+        o += wgt * wo[(w * MT + m) * HD + d];
+      }
+    }
+    p.part_o[(part * p.M + m) * HD + d] = o;
+    if (d == 0) {
+      p.part_ml[(part * p.M + m) * 2] = mx;
+      p.part_ml[(part * p.M + m) * 2 + 1] = l;
+    }
+  }
+}
+
+// o[b, m, h, :] = sum_s 2^(m_s - mx) o_s / sum_s 2^(m_s - mx) l_s ;  lse = ln2 * (mx + log2 L).
+// One CTA of HD threads per (b, h, m).  Split 0 holds key 0, visible to every query, so
+// mx is finite.
+__global__ void __launch_bounds__(HD) decode_combine_kernel(const float* part_o, const float* part_ml,
+                                                            __nv_bfloat16* o, float* lse, int M, int H, int S) {
+  const int m = (int)(blockIdx.x % M);
+  const int bh = (int)(blockIdx.x / M);
+  const int h = bh % H, b = bh / H;
+  const int d = threadIdx.x;
+  const float* ml = part_ml + (size_t)bh * S * M * 2;
+  float mx = -INFINITY;
+  for (int s = 0; s < S; ++s) mx = fmaxf(mx, ml[(s * M + m) * 2]);
+  float L = 0.0f, acc = 0.0f;
+  for (int s = 0; s < S; ++s) {
+    const float ms = ml[(s * M + m) * 2];
+    if (ms == -INFINITY) continue;
+    const float w = exp2f(ms - mx);
+    L += w * ml[(s * M + m) * 2 + 1];
+    acc += w * part_o[(((size_t)bh * S + s) * M + m) * HD + d];
+  }
+  o[((size_t)(b * M + m) * H + h) * HD + d] = __float2bfloat16_rn(acc / L);
+  if (d == 0) lse[(size_t)bh * M + m] = (mx + log2f(L)) * 0.69314718055994531f;
+}
+
+template <int MT>
+cudaError_t launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const Params& p, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const long long grid = (long long)p.B * p.H * p.S;
+  decode_split_kernel<MT><<<(unsigned)grid, NTHREADS, SMEM_BYTES, st>>>(tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace dec
+
+int decode_splits(int B, int N, int H, int n_sm, int* tiles_per_split) {
+  const int n_tiles = (N + dec::TK - 1) / dec::TK;
+  const long long units = (long long)B * H;
+  const long long base_ctas = units * ((n_tiles + 7) / 8);  // about 8 tiles (1024 keys) per CTA
+  const long long waves = (base_ctas + n_sm - 1) / n_sm;
+  long long s = (waves * n_sm) / units;
+  if (s < 1) s = 1;
+  if (s > n_tiles) s = n_tiles;
+  if (s > kDecodeMaxSplits) s = kDecodeMaxSplits;
+  const int tps = (int)((n_tiles + s - 1) / s);
+  *tiles_per_split = tps;
+  return (n_tiles + tps - 1) / tps;
+}
+
+cudaError_t launch_decode_sm100(const CUtensorMap& tk, const CUtensorMap& tv, const void* q, void* o, float* lse,
+                                float* part_o, float* part_ml, int B, int M, int N, int H, int S,
+                                int tiles_per_split, int* err, cudaStream_t st) {
+  dec::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.part_o = part_o;
+  p.part_ml = part_ml;
+  p.B = B;
+  p.M = M;
+  p.N = N;
+  p.H = H;
+  p.S = S;
+  p.tiles_per_split = tiles_per_split;
+  p.qscale = (float)(1.4426950408889634 / sqrt((double)dec::HD));
+  p.err = err;
+  const long long grid = (long long)B * H * S;
+  if (grid <= 0 || grid > 0x7fffffffLL || M < 1 || M > dec::MAXM) return cudaErrorInvalidValue;
+  cudaError_t e;
+  if (M == 1) e = dec::launch_split<1>(tk, tv, p, st);
+  else if (M == 2) e = dec::launch_split<2>(tk, tv, p, st);
+  else if (M <= 4) e = dec::launch_split<4>(tk, tv, p, st);
+  else if (M <= 8) e = dec::launch_split<8>(tk, tv, p, st);
+  else e = dec::launch_split<16>(tk, tv, p, st);
+  if (e != cudaSuccess) return e;
+  const long long cgrid = (long long)B * H * M;
+  dec::decode_combine_kernel<<<(unsigned)cgrid, dec::HD, 0, st>>>(part_o, part_ml, static_cast<__nv_bfloat16*>(o),
+                                                                  lse, M, H, S);
+  return cudaGetLastError();
+}
+
+}  // namespace s2

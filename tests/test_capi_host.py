@@ -27,7 +27,8 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for required in ("s2attn_fwd", "s2attn_bwd", "rope_pi_apply", "s2attn_bwd_workspace_bytes",
-                     "s2attn_fwd_f32", "s2attn_bwd_f32", "s2attn_get_device_error"):
+                     "s2attn_fwd_f32", "s2attn_bwd_f32", "s2attn_get_device_error", "s2attn_decode",
+                     "s2attn_decode_workspace_bytes"):
         assert required in names
 
 
@@ -85,6 +86,29 @@ def test_rope_validation(lib):
     p = ctypes.c_void_p(0x1000)
     assert lib.rope_pi_apply(p, NULL, 1, 16, 2, 100, 0.5, 10000.0, NULL) == -1      # D % 16 != 0
     assert lib.rope_pi_apply(p, NULL, 1, 16, 2, 128, 0.5, -1.0, NULL) == -1         # bad base
+
+
+@pytest.mark.parametrize("args,status", [
+    ((1, 0, 100, 2, 128), -1),     # no query
+    ((1, 5, 4, 2, 128), -1),       # more queries than positions
+    ((0, 1, 100, 2, 128), -1),     # empty batch
+    ((1, 17, 100, 2, 128), -2),    # more than 16 queries
+    ((1, 1, 100, 2, 64), -2),      # D = 64
+    ((1, 1, 100, 2, 128), -1),     # valid shape, null pointers
+])
+def test_decode_validation(lib, args, status):
+    assert lib.s2attn_decode(NULL, NULL, NULL, NULL, NULL, *args, NULL, 0, NULL) == status
+
+
+def test_decode_workspace_size(lib):
+    # fp32 partials per (b, h, split, query): D output values + (max, sum); at most one split
+    # per 128-key tile and at most 64 splits
+    B, M, N, H, D = 1, 4, 32768, 32, 128
+    assert lib.s2attn_decode_workspace_bytes(B, M, N, H, D) == B * H * 64 * M * (D + 2) * 4
+    assert lib.s2attn_decode_workspace_bytes(1, 1, 200, 2, 128) == 2 * 2 * 128 * 4 + 256
+    assert lib.s2attn_decode_workspace_bytes(1, 2, 1, 2, 128) == 0
+    p = ctypes.c_void_p(0x10000)
+    assert lib.s2attn_decode(p, p, p, p, p, B, M, N, H, D, p, 1024, NULL) == -3
 
 
 def test_workspace_checked_before_launch(lib):
