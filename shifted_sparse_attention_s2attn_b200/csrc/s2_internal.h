@@ -42,12 +42,13 @@ cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const
                            cudaStream_t st);
 
 // Decoding step (full causal attention of the last M <= 16 positions), D == 128.
-// The K/V of each (b, h) is cut into `S` splits of `tiles_per_split` 128-key tiles
+// The K/V of each (b, h) is cut into `S` splits of `tiles_per_split` key tiles
 // (decode_splits picks them for `n_sm` SMs, at most kDecodeMaxSplits); the split kernel
 // writes fp32 partials (part_o [B*H][S][M][128], part_ml [B*H][S][M][2]) and a second
-// kernel combines them into o and lse.  Tensor maps: 128-row boxes of 64 columns,
+// kernel combines them into o and lse.  Tensor maps: 64-row boxes of 64 columns,
 // 128-byte swizzle, over k and v ([B,N,H,D]).
 constexpr int kDecodeMaxSplits = 64;
+constexpr int kDecodeTileKeys = 64;
 int decode_splits(int B, int N, int H, int n_sm, int* tiles_per_split);
 cudaError_t launch_decode_sm100(const CUtensorMap& tk, const CUtensorMap& tv, const void* q, void* o, float* lse,
                                 float* part_o, float* part_ml, int B, int M, int N, int H, int S,

@@ -198,10 +198,10 @@ int check_decode_shape(int B, int M, int N, int H, int D) {
   return S2ATTN_OK;
 }
 
-// Splits the workspace is sized for: the most any device can get (1 per 128-key tile,
+// Splits the workspace is sized for: the most any device can get (1 per key tile,
 // at most kDecodeMaxSplits), so that the size does not depend on the device.
 int decode_max_splits(int N) {
-  const int tiles = (N + 127) / 128;
+  const int tiles = (N + s2::kDecodeTileKeys - 1) / s2::kDecodeTileKeys;
   return tiles < s2::kDecodeMaxSplits ? tiles : s2::kDecodeMaxSplits;
 }
 
@@ -321,7 +321,8 @@ int s2attn_decode(const void* q, const void* k, const void* v, void* o, float* l
   float* part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_part_o_bytes(B, M, N, H, D));
   const s2::Shape s{B, N, H, D, N, 0};
   CUtensorMap tk, tv;
-  if (!map_bf16_sw128(&tk, k, s, 128) || !map_bf16_sw128(&tv, v, s, 128)) return S2ATTN_ERR_CUDA;
+  if (!map_bf16_sw128(&tk, k, s, s2::kDecodeTileKeys) || !map_bf16_sw128(&tv, v, s, s2::kDecodeTileKeys))
+    return S2ATTN_ERR_CUDA;
   int* err = error_word_ptr();
   if (!err) return S2ATTN_ERR_CUDA;
   return cuda_status(s2::launch_decode_sm100(tk, tv, q, o, lse, part_o, part_ml, B, M, N, H, S, tps, err,

@@ -10,13 +10,16 @@
 // every head: 2*N*D*2 bytes per head and 4*M*D FLOPs per key, so it is bound by HBM, not
 // by arithmetic -- it runs on the CUDA cores, and its job is to stream K and V at full
 // bandwidth:
-//   * split-KV: CTA (b, h, split) takes a run of 128-key tiles of one head, so that the
-//     grid fills every SM even for one sequence (B*H*splits CTAs);
-//   * a producer thread streams the tiles with TMA (four 128-row x 64-column boxes per
-//     tile: K and V, two column halves each, 128-byte swizzle) through a 3-stage ring;
-//   * 4 consumer warps take 32 keys of each tile: lane = key for Q.K (16-byte swizzled
-//     row reads, conflict-free), an online base-2 softmax per warp, then lane = 4 head
-//     dims for P.V (the probabilities broadcast from shared memory);
+//   * split-KV: CTA (b, h, split) takes a run of 64-key tiles of one head, so that the
+//     grid fills every SM even for one sequence (B*H*splits CTAs, sized to whole waves);
+//   * a producer thread streams the tiles with TMA (four 64-row x 64-column boxes per
+//     tile: K and V, two column halves each, 128-byte swizzle) through a 3-stage ring,
+//     starting before the queries are staged; two CTAs fit on an SM, so one CTA's
+//     start-up and merge overlap the other's streaming;
+//   * consumer warps take 32 keys of each tile (and, for more than 8 queries, half of
+//     the queries): lane = key for Q.K (16-byte swizzled row reads, conflict-free), an
+//     online base-2 softmax per warp, then lane = 4 head dims for P.V (the
+//     probabilities broadcast from shared memory);
 //   * the warps' partial (max, sum, unnormalised output) merge in shared memory and the
 //     CTA writes one fp32 partial per (b, h, split, m); a second kernel combines the
 //     splits into o (bf16) and lse.
@@ -27,18 +30,25 @@ namespace s2 {
 namespace dec {
 
 constexpr int HD = 128;
-constexpr int TK = 128;                       // keys per tile
-constexpr uint32_t BOX = TK * 128;            // 128 rows x 128 B (64 bf16 columns)
+constexpr int TK = kDecodeTileKeys;          // keys per tile (64; the tensor maps' box height)
+constexpr uint32_t BOX = TK * 128;            // 64 rows x 128 B (64 bf16 columns)
 constexpr uint32_t TILE_BYTES = 4 * BOX;      // K box 0, K box 1, V box 0, V box 1
 constexpr int NST = 3;                        // ring stages
 constexpr int MAXM = 16;
-constexpr int NCW = 4;                        // consumer warps
-constexpr int NTHREADS = (NCW + 1) * 32;      // + producer warp
+constexpr int KW = TK / 32;                   // key warps: 32 keys of each tile per warp
+constexpr int MAXW = 2 * KW;                  // consumer warps with the queries split in two
 constexpr uint32_t OFF_Q = NST * TILE_BYTES;              // float [MAXM][HD], scaled to the log2 domain
-constexpr uint32_t OFF_P = OFF_Q + MAXM * HD * 4;         // float [NCW][32 keys][MT]
-constexpr uint32_t OFF_BAR = OFF_P + NCW * 32 * MAXM * 4;
+constexpr uint32_t OFF_P = OFF_Q + MAXM * HD * 4;         // float [warp][32 keys][queries of the warp]
+constexpr uint32_t OFF_BAR = OFF_P + MAXW * 32 * 8 * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + 2 * NST * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;     // + slack to align the base to 1024 B
+static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs must fit on an SM");
+// Queries per consumer warp and consumer warps, for a query count padded to MT.
+template <int MT> struct Cfg {
+  static constexpr int QW = MT > 8 ? 8 : MT;
+  static constexpr int NCW = KW * (MT / QW);
+  static constexpr int NTHREADS = (NCW + 1) * 32;  // + producer warp
+};
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct Params {
@@ -73,9 +83,10 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 template <int MT>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                         const Params p) {
+  constexpr int QW = Cfg<MT>::QW, NCW = Cfg<MT>::NCW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -84,8 +95,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float* qs = reinterpret_cast<float*>(smem + OFF_Q);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int split = (int)(blockIdx.x % p.S);
-  const int bh = (int)(blockIdx.x / p.S);
+  // consecutive CTAs take the same split of consecutive heads: the CTAs resident at one
+  // time then read whole [H, D] token rows (8 KB at H = 32) rather than one head's 256 B
+  // of each, so every DRAM page they open is read in full
+  const int units = p.B * p.H;
+  const int bh = (int)(blockIdx.x % units);
+  const int split = (int)(blockIdx.x / units);
   const int h = bh % p.H, b = bh / p.H;
   const int t_begin = split * p.tiles_per_split * TK;
   const int t_end = min(p.N, t_begin + p.tiles_per_split * TK);
@@ -98,16 +113,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     *abort_flag = (*(volatile int*)p.err != 0) ? 1 : 0;
     fence_mbar_init();
-  }
-  // queries of this head, scaled into the log2 domain; rows m >= M are zero
-  if (threadIdx.x < HD) {
-    const int d = threadIdx.x;
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      float x = 0.0f;
-      if (m < p.M) x = __bfloat162float(p.q[((size_t)(b * p.M + m) * p.H + h) * HD + d]) * p.qscale;
-      qs[m * HD + d] = x;
-    }
   }
   __syncthreads();
   const bool skip = *abort_flag != 0;
@@ -144,18 +149,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     return;  // the producer warp takes no part in the merge below
   }
 
-  // ---------------- consumers: 32 keys of each tile per warp ----------------
-  float m_run[MT], l_lane[MT], o_acc[MT][4];
+  // ---------------- consumers: 32 keys of each tile and QW queries per warp ----------------
+  // queries of this head, scaled into the log2 domain; rows m >= M are zero (the
+  // producer's first copies are already in flight)
+  for (int i = threadIdx.x; i < MT * HD; i += NCW * 32) {
+    const int m = i / HD, d = i % HD;
+    float x = 0.0f;
+    if (m < p.M) x = __bfloat162float(p.q[((size_t)(b * p.M + m) * p.H + h) * HD + d]) * p.qscale;
+    qs[i] = x;
+  }
+  named_bar_sync(1, NCW * 32);
+  const int kw = warp % KW;          // which 32 keys of each tile
+  const int q0 = (warp / KW) * QW;   // first query of this warp
+  float m_run[QW], l_lane[QW], o_acc[QW][4];
 #pragma unroll
-  for (int m = 0; m < MT; ++m) {
+  for (int m = 0; m < QW; ++m) {
     m_run[m] = -INFINITY;
     l_lane[m] = 0.0f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) o_acc[m][e] = 0.0f;
   }
-  const float4* q4 = reinterpret_cast<const float4*>(qs);
-  float* pbuf = reinterpret_cast<float*>(smem + OFF_P) + warp * 32 * MT;
-  const int lim0 = p.N - p.M;  // query m sees keys t <= lim0 + m
+  const float4* q4 = reinterpret_cast<const float4*>(qs + q0 * HD);
+  float* pbuf = reinterpret_cast<float*>(smem + OFF_P) + warp * 32 * QW;
+  const int lim0 = p.N - p.M + q0;  // query q0 + m sees keys t <= lim0 + m
   bool ok = !skip;
   for (int i = 0; i < n_tiles && ok; ++i) {
     const int slot = i % NST;
@@ -163,20 +179,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!ok) break;
     const uint8_t* kb = smem + slot * TILE_BYTES;
     const uint8_t* vb = kb + 2 * BOX;
-    const int t0 = t_begin + i * TK + 32 * warp;  // first key of this warp's 32
+    const int t0 = t_begin + i * TK + 32 * kw;  // first key of this warp's 32
     // ---- scores, lane = key: s_m = (q_m * log2e / sqrt(D)) . k_t
-    const int r = 32 * warp + lane;
+    const int r = 32 * kw + lane;
     const int t = t0 + lane;
-    float s[MT];
+    float s[QW];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) s[m] = 0.0f;
+    for (int m = 0; m < QW; ++m) s[m] = 0.0f;
 #pragma unroll 4
     for (int c = 0; c < HD / 8; ++c) {
       const uint4 kw = *reinterpret_cast<const uint4*>(kb + (c >> 3) * BOX + r * 128 + (((c & 7) ^ (r & 7)) << 4));
       float kf[8];
       bf16x8_to_f32(kw, kf);
 #pragma unroll
-      for (int m = 0; m < MT; ++m) {
+      for (int m = 0; m < QW; ++m) {
         const float4 qa = q4[(m * HD + 8 * c) / 4], qb = q4[(m * HD + 8 * c) / 4 + 1];
         float a = s[m];
         a = fmaf(qa.x, kf[0], a);
@@ -193,7 +209,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // ---- online softmax over this warp's 32 keys (keys past the split or the causal
     // limit of query m count as -inf)
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
+    for (int m = 0; m < QW; ++m) {
       const bool vis = t < t_end && t <= lim0 + m;
       const float sm = vis ? s[m] : -INFINITY;
       const float m_new = fmaxf(m_run[m], warp_max(sm));
@@ -209,7 +225,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         pr = vis ? ex2_approx(sm - m_new) : 0.0f;
       }
       l_lane[m] += pr;
-      pbuf[lane * MT + m] = pr;
+      pbuf[lane * QW + m] = pr;
     }
     __syncwarp();
     // ---- o += p . v, lane = head dims [4*lane, 4*lane + 4)
@@ -217,14 +233,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t vcol = (lane >> 4) * BOX + (lane & 1) * 8;
     const int vchunk = (lane & 15) >> 1;
     for (int j = 0; j < nv; ++j) {
-      const int rr = 32 * warp + j;
+      const int rr = 32 * kw + j;
       const uint2 vw = *reinterpret_cast<const uint2*>(vb + vcol + rr * 128 + ((vchunk ^ (rr & 7)) << 4));
       const float v0 = __uint_as_float(vw.x << 16), v1 = __uint_as_float(vw.x & 0xffff0000u);
       const float v2 = __uint_as_float(vw.y << 16), v3 = __uint_as_float(vw.y & 0xffff0000u);
-      const float* pj = pbuf + j * MT;
-      if constexpr (MT >= 4) {
+      const float* pj = pbuf + j * QW;
+      if constexpr (QW >= 4) {
 #pragma unroll
-        for (int m = 0; m < MT; m += 4) {
+        for (int m = 0; m < QW; m += 4) {
           const float4 p4 = *reinterpret_cast<const float4*>(pj + m);
           const float pm[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
@@ -237,7 +253,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       } else {
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
+        for (int m = 0; m < QW; ++m) {
           const float pm = pj[m];
           o_acc[m][0] = fmaf(pm, v0, o_acc[m][0]);
           o_acc[m][1] = fmaf(pm, v1, o_acc[m][1]);
@@ -254,33 +270,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     *abort_flag = 1;
   }
 
-  // ---------------- merge the 4 warps' partials (consumer threads only) ----------------
+  // ---------------- merge the key warps' partials (consumer threads only) ----------------
   // Every tile has been consumed, so no copy is in flight and the ring's memory is free.
+  // Query q0 + m of warp w goes to slot (kw, q0 + m).
   named_bar_sync(1, NCW * 32);
-  float* wo = reinterpret_cast<float*>(smem);                 // [NCW][MT][HD]
-  float* wml = wo + NCW * MT * HD;                            // [NCW][MT][2]
+  float* wo = reinterpret_cast<float*>(smem);                 // [KW][MT][HD]
+  float* wml = wo + KW * MT * HD;                             // [KW][MT][2]
 #pragma unroll
-  for (int m = 0; m < MT; ++m) {
+  for (int m = 0; m < QW; ++m) {
     const float l = warp_sum(l_lane[m]);
-    *reinterpret_cast<float4*>(wo + (warp * MT + m) * HD + 4 * lane) =
+    *reinterpret_cast<float4*>(wo + (kw * MT + q0 + m) * HD + 4 * lane) =
         make_float4(o_acc[m][0], o_acc[m][1], o_acc[m][2], o_acc[m][3]);
     if (lane == 0) {
-      wml[(warp * MT + m) * 2] = m_run[m];
-      wml[(warp * MT + m) * 2 + 1] = l;
+      wml[(kw * MT + q0 + m) * 2] = m_run[m];
+      wml[(kw * MT + q0 + m) * 2 + 1] = l;
     }
   }
   named_bar_sync(1, NCW * 32);
   if (skip || *abort_flag) return;
-  const int d = threadIdx.x;  // 0 .. 127
   const size_t part = (size_t)bh * p.S + split;
-  for (int m = 0; m < p.M; ++m) {
+  for (int i = threadIdx.x; i < p.M * HD; i += NCW * 32) {
+    const int m = i / HD, d = i % HD;
     float mx = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, wml[(w * MT + m) * 2]);
+    for (int w = 0; w < KW; ++w) mx = fmaxf(mx, wml[(w * MT + m) * 2]);
     float l = 0.0f, o = 0.0f;
     if (mx != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < NCW; ++w) {
+      for (int w = 0; w < KW; ++w) {
         const float wm = wml[(w * MT + m) * 2];
         const float wgt = ex2_approx(wm - mx);  // 0 for a warp that saw no visible key
         l += wgt * wml[(w * MT + m) * 2 + 1];
@@ -325,7 +342,7 @@ cudaError_t launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const Par
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const long long grid = (long long)p.B * p.H * p.S;
-  decode_split_kernel<MT><<<(unsigned)grid, NTHREADS, SMEM_BYTES, st>>>(tk, tv, p);
+  decode_split_kernel<MT><<<(unsigned)grid, Cfg<MT>::NTHREADS, SMEM_BYTES, st>>>(tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -334,9 +351,10 @@ cudaError_t launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const Par
 int decode_splits(int B, int N, int H, int n_sm, int* tiles_per_split) {
   const int n_tiles = (N + dec::TK - 1) / dec::TK;
   const long long units = (long long)B * H;
-  const long long base_ctas = units * ((n_tiles + 7) / 8);  // about 8 tiles (1024 keys) per CTA
-  const long long waves = (base_ctas + n_sm - 1) / n_sm;
-  long long s = (waves * n_sm) / units;
+  const long long slots = 2LL * n_sm;                          // two CTAs per SM
+  const long long base_ctas = units * ((n_tiles + 15) / 16);  // about 16 tiles (1024 keys) per CTA
+  const long long waves = (base_ctas + slots - 1) / slots;
+  long long s = (waves * slots) / units;
   if (s < 1) s = 1;
   if (s > n_tiles) s = n_tiles;
   if (s > kDecodeMaxSplits) s = kDecodeMaxSplits;

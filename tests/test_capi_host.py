@@ -102,10 +102,10 @@ def test_decode_validation(lib, args, status):
 
 def test_decode_workspace_size(lib):
     # fp32 partials per (b, h, split, query): D output values + (max, sum); at most one split
-    # per 128-key tile and at most 64 splits
+    # per 64-key tile and at most 64 splits
     B, M, N, H, D = 1, 4, 32768, 32, 128
     assert lib.s2attn_decode_workspace_bytes(B, M, N, H, D) == B * H * 64 * M * (D + 2) * 4
-    assert lib.s2attn_decode_workspace_bytes(1, 1, 200, 2, 128) == 2 * 2 * 128 * 4 + 256
+    assert lib.s2attn_decode_workspace_bytes(1, 1, 200, 2, 128) == 2 * 4 * 128 * 4 + 256
     assert lib.s2attn_decode_workspace_bytes(1, 2, 1, 2, 128) == 0
     p = ctypes.c_void_p(0x10000)
     assert lib.s2attn_decode(p, p, p, p, p, B, M, N, H, D, p, 1024, NULL) == -3
