@@ -23,6 +23,8 @@
 //   * the warps' partial (max, sum, unnormalised output) merge in shared memory and the
 //     CTA writes one fp32 partial per (b, h, split, m); a second kernel combines the
 //     splits into o (bf16) and lse.
+#include <atomic>
+
 #include "s2_internal.h"
 #include "s2_ptx.cuh"
 
@@ -116,6 +118,9 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 2)
   }
   __syncthreads();
   const bool skip = *abort_flag != 0;
+  // the combine kernel may be scheduled now; it waits for this whole grid to finish
+  // (griddepcontrol.wait) before it reads anything this grid writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == NCW) {
     // ---------------- TMA producer ----------------
@@ -313,34 +318,73 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 2)
 }
 
 // o[b, m, h, :] = sum_s 2^(m_s - mx) o_s / sum_s 2^(m_s - mx) l_s ;  lse = ln2 * (mx + log2 L).
-// One CTA of HD threads per (b, h, m).  Split 0 holds key 0, visible to every query, so
-// mx is finite.
+// One CTA of HD threads per (b, h, m).  The splits' (max, sum) pairs are loaded in one
+// parallel round into shared memory, and each thread's loads of its column of the S
+// partial outputs are independent, so the step costs a few memory latencies instead of
+// one per split.  Split 0 holds key 0, visible to every query, so mx is finite.
 __global__ void __launch_bounds__(HD) decode_combine_kernel(const float* part_o, const float* part_ml,
                                                             __nv_bfloat16* o, float* lse, int M, int H, int S) {
+  static_assert(kDecodeMaxSplits <= HD, "one thread per split");
+  __shared__ float wgt[kDecodeMaxSplits];
+  __shared__ float red[HD / 32];
   const int m = (int)(blockIdx.x % M);
   const int bh = (int)(blockIdx.x / M);
   const int h = bh % H, b = bh / H;
-  const int d = threadIdx.x;
+  const int d = threadIdx.x, warp = d / 32, lane = d % 32;
+  // launched as a programmatic dependent of the split kernel: wait until that grid has
+  // completed and its writes are visible (a no-op under ordinary stream order)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const float* ml = part_ml + (size_t)bh * S * M * 2;
-  float mx = -INFINITY;
-  for (int s = 0; s < S; ++s) mx = fmaxf(mx, ml[(s * M + m) * 2]);
-  float L = 0.0f, acc = 0.0f;
-  for (int s = 0; s < S; ++s) {
-    const float ms = ml[(s * M + m) * 2];
-    if (ms == -INFINITY) continue;
-    const float w = exp2f(ms - mx);
-    L += w * ml[(s * M + m) * 2 + 1];
-    acc += w * part_o[(((size_t)bh * S + s) * M + m) * HD + d];
+  const float ms = d < S ? ml[(d * M + m) * 2] : -INFINITY;
+  const float ls = d < S ? ml[(d * M + m) * 2 + 1] : 0.0f;
+  // mx = max over splits (thread d holds split d; S <= kDecodeMaxSplits <= HD)
+  float x = ms;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
+  if (lane == 0) red[warp] = x;
+  __syncthreads();
+  float mx = red[0];
+#pragma unroll
+  for (int w = 1; w < HD / 32; ++w) mx = fmaxf(mx, red[w]);
+  __syncthreads();
+  const float w_s = (d < S && ms != -INFINITY) ? exp2f(ms - mx) : 0.0f;
+  if (d < S) wgt[d] = w_s;
+  float y = w_s * ls;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
+  if (lane == 0) red[warp] = y;
+  __syncthreads();
+  float L = 0.0f;
+#pragma unroll
+  for (int w = 0; w < HD / 32; ++w) L += red[w];
+  const float* po = part_o + ((size_t)bh * S * M + m) * HD + d;  // split s at po[s * M * HD]
+  float acc = 0.0f;
+  int sidx = 0;
+  for (; sidx + 8 <= S; sidx += 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = po[(size_t)(sidx + u) * M * HD];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc = fmaf(wgt[sidx + u], v[u], acc);
   }
+  for (; sidx < S; ++sidx) acc = fmaf(wgt[sidx], po[(size_t)sidx * M * HD], acc);
   o[((size_t)(b * M + m) * H + h) * HD + d] = __float2bfloat16_rn(acc / L);
   if (d == 0) lse[(size_t)bh * M + m] = (mx + log2f(L)) * 0.69314718055994531f;
 }
 
 template <int MT>
 cudaError_t launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const Params& p, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
+  // the shared-memory limit is a per-device function attribute: set it once per device
+  static std::atomic<uint64_t> done_mask{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (!bit || !(done_mask.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(decode_split_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  }
   const long long grid = (long long)p.B * p.H * p.S;
   decode_split_kernel<MT><<<(unsigned)grid, Cfg<MT>::NTHREADS, SMEM_BYTES, st>>>(tk, tv, p);
   return cudaGetLastError();
@@ -387,10 +431,20 @@ cudaError_t launch_decode_sm100(const CUtensorMap& tk, const CUtensorMap& tv, co
   else if (M <= 8) e = dec::launch_split<8>(tk, tv, p, st);
   else e = dec::launch_split<16>(tk, tv, p, st);
   if (e != cudaSuccess) return e;
-  const long long cgrid = (long long)B * H * M;
-  dec::decode_combine_kernel<<<(unsigned)cgrid, dec::HD, 0, st>>>(part_o, part_ml, static_cast<__nv_bfloat16*>(o),
-                                                                  lse, M, H, S);
-  return cudaGetLastError();
+  // the combine kernel is a programmatic dependent launch: it is scheduled while the
+  // split kernel drains, which hides its launch latency
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long long)B * H * M));
+  cfg.blockDim = dim3(dec::HD);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, dec::decode_combine_kernel, static_cast<const float*>(part_o),
+                            static_cast<const float*>(part_ml), static_cast<__nv_bfloat16*>(o), lse, M, H, S);
 }
 
 }  // namespace s2
