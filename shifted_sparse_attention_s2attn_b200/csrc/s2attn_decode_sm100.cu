@@ -51,7 +51,6 @@ template <int MT> struct Cfg {
   static constexpr int NCW = KW * (MT / QW);
   static constexpr int NTHREADS = (NCW + 1) * 32;  // + producer warp
 };
-constexpr float LOG2E = 1.4426950408889634f;
 
 struct Params {
   const __nv_bfloat16* q;
