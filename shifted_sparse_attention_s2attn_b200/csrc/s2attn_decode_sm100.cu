@@ -317,58 +317,74 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 2)
 }
 
 // o[b, m, h, :] = sum_s 2^(m_s - mx) o_s / sum_s 2^(m_s - mx) l_s ;  lse = ln2 * (mx + log2 L).
-// One CTA of HD threads per (b, h, m).  The splits' (max, sum) pairs are loaded in one
-// parallel round into shared memory, and each thread's loads of its column of the S
-// partial outputs are independent, so the step costs a few memory latencies instead of
-// one per split.  Split 0 holds key 0, visible to every query, so mx is finite.
-__global__ void __launch_bounds__(HD) decode_combine_kernel(const float* part_o, const float* part_ml,
-                                                            __nv_bfloat16* o, float* lse, int M, int H, int S) {
-  static_assert(kDecodeMaxSplits <= HD, "one thread per split");
+// One CTA per (b, h, m) with CG groups of HD threads: the splits' (max, sum) pairs are loaded
+// in one parallel round, and group g sums splits g, g+CG, ... of its column d with
+// independent loads, so the step costs about two memory latencies.  Split 0 holds key 0,
+// visible to every query, so mx is finite.
+constexpr int CG = 4;
+__global__ void __launch_bounds__(CG * HD) decode_combine_kernel(const float* part_o, const float* part_ml,
+                                                                 __nv_bfloat16* o, float* lse, int M, int H,
+                                                                 int S) {
+  static_assert(kDecodeMaxSplits <= HD, "the first HD threads hold one split each");
   __shared__ float wgt[kDecodeMaxSplits];
-  __shared__ float red[HD / 32];
+  __shared__ float red[HD / 32][2];
+  __shared__ float part[CG][HD];
   const int m = (int)(blockIdx.x % M);
   const int bh = (int)(blockIdx.x / M);
   const int h = bh % H, b = bh / H;
-  const int d = threadIdx.x, warp = d / 32, lane = d % 32;
+  const int tid = threadIdx.x, grp = tid / HD, d = tid % HD, warp = tid / 32, lane = tid % 32;
   // launched as a programmatic dependent of the split kernel: wait until that grid has
   // completed and its writes are visible (a no-op under ordinary stream order)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float* ml = part_ml + (size_t)bh * S * M * 2;
-  const float ms = d < S ? ml[(d * M + m) * 2] : -INFINITY;
-  const float ls = d < S ? ml[(d * M + m) * 2 + 1] : 0.0f;
-  // mx = max over splits (thread d holds split d; S <= kDecodeMaxSplits <= HD)
+  // group 0: thread d holds split d; mx = max over splits, L = sum of weighted sums
+  float ms = -INFINITY, ls = 0.0f;
+  if (grp == 0 && d < S) {
+    ms = ml[(d * M + m) * 2];
+    ls = ml[(d * M + m) * 2 + 1];
+  }
   float x = ms;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, off));
-  if (lane == 0) red[warp] = x;
+  if (grp == 0 && lane == 0) red[warp][0] = x;
   __syncthreads();
-  float mx = red[0];
+  float mx = red[0][0];
 #pragma unroll
-  for (int w = 1; w < HD / 32; ++w) mx = fmaxf(mx, red[w]);
-  __syncthreads();
-  const float w_s = (d < S && ms != -INFINITY) ? exp2f(ms - mx) : 0.0f;
-  if (d < S) wgt[d] = w_s;
+  for (int w = 1; w < HD / 32; ++w) mx = fmaxf(mx, red[w][0]);
+  const float w_s = (grp == 0 && d < S && ms != -INFINITY) ? exp2f(ms - mx) : 0.0f;
+  if (grp == 0 && d < S) wgt[d] = w_s;
   float y = w_s * ls;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
-  if (lane == 0) red[warp] = y;
+  if (grp == 0 && lane == 0) red[warp][1] = y;
   __syncthreads();
-  float L = 0.0f;
-#pragma unroll
-  for (int w = 0; w < HD / 32; ++w) L += red[w];
+  // group grp: splits grp, grp + CG, ... (at most kDecodeMaxSplits / CG = 16), loads first
   const float* po = part_o + ((size_t)bh * S * M + m) * HD + d;  // split s at po[s * M * HD]
-  float acc = 0.0f;
-  int sidx = 0;
-  for (; sidx + 8 <= S; sidx += 8) {
-    float v[8];
+  constexpr int PER = kDecodeMaxSplits / CG;
+  float v[PER];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = po[(size_t)(sidx + u) * M * HD];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) acc = fmaf(wgt[sidx + u], v[u], acc);
+  for (int u = 0; u < PER; ++u) {
+    const int sidx = grp + u * CG;
+    v[u] = sidx < S ? po[(size_t)sidx * M * HD] : 0.0f;
   }
-  for (; sidx < S; ++sidx) acc = fmaf(wgt[sidx], po[(size_t)sidx * M * HD], acc);
-  o[((size_t)(b * M + m) * H + h) * HD + d] = __float2bfloat16_rn(acc / L);
-  if (d == 0) lse[(size_t)bh * M + m] = (mx + log2f(L)) * 0.69314718055994531f;
+  float acc = 0.0f;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int sidx = grp + u * CG;
+    if (sidx < S) acc = fmaf(wgt[sidx], v[u], acc);
+  }
+  part[grp][d] = acc;
+  __syncthreads();
+  if (grp == 0) {
+    float L = 0.0f;
+#pragma unroll
+    for (int w = 0; w < HD / 32; ++w) L += red[w][1];
+    float tot = 0.0f;
+#pragma unroll
+    for (int g = 0; g < CG; ++g) tot += part[g][d];
+    o[((size_t)(b * M + m) * H + h) * HD + d] = __float2bfloat16_rn(tot / L);
+    if (d == 0) lse[(size_t)bh * M + m] = (mx + log2f(L)) * 0.69314718055994531f;
+  }
 }
 
 template <int MT>
@@ -434,7 +450,7 @@ cudaError_t launch_decode_sm100(const CUtensorMap& tk, const CUtensorMap& tv, co
   // split kernel drains, which hides its launch latency
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((long long)B * H * M));
-  cfg.blockDim = dim3(dec::HD);
+  cfg.blockDim = dim3(dec::CG * dec::HD);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
