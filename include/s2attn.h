@@ -109,7 +109,9 @@ int s2attn_bwd_dq_convert(const float* dq_acc, void* dq, int B, int N, int H, in
  *   o    : [B,M,H,D] bf16 output; query m attends to the keys at positions
  *          0 .. N-M+m with scale 1/sqrt(D)
  *   lse  : [B,H,M] fp32 output, natural log of sum over those keys of exp(scale*q.k)
- * Requirements: 1 <= M <= N; M <= 16 and D == 128 (else S2ATTN_ERR_UNSUPPORTED).
+ * Requirements: 1 <= M <= N; M <= 128 and D == 128 (else S2ATTN_ERR_UNSUPPORTED).
+ * One query runs on CUDA cores (HBM-bound matrix-vector work); 2..128 queries run one
+ * 128-row query tile on the tensor cores (speculative decoding, chunked prefill).
  * `workspace` (device, caller-owned, 256-byte aligned, at least
  * s2attn_decode_workspace_bytes bytes) receives per-split partial results and is
  * overwritten.  V rows past a query's causal limit are multiplied by a zero weight,

@@ -41,14 +41,25 @@ cudaError_t launch_bwd_f32(const float* q, const float* k, const float* v, const
                            const float* lse, float* dq, float* dk, float* dv, float* delta, const Shape& s,
                            cudaStream_t st);
 
-// Decoding step (full causal attention of the last M <= 16 positions), D == 128.
+// Decoding step (full causal attention of the last M <= 128 positions), D == 128; the
+// CUDA-core kernel below takes M <= kDecodeSimtMaxM.
 // The K/V of each (b, h) is cut into `S` splits of `tiles_per_split` key tiles
 // (decode_splits picks them for `n_sm` SMs, at most kDecodeMaxSplits); the split kernel
 // writes fp32 partials (part_o [B*H][S][M][128], part_ml [B*H][S][M][2]) and a second
 // kernel combines them into o and lse.  Tensor maps: 64-row boxes of 64 columns,
 // 128-byte swizzle, over k and v ([B,N,H,D]).
 constexpr int kDecodeMaxSplits = 64;
-constexpr int kDecodeTileKeys = 64;
+constexpr int kDecodeTileKeys = 64;       // key tile of the CUDA-core kernel (its tensor maps' box height)
+// Up to this many queries the CUDA-core kernel runs, above it the tensor-core one (measured at
+// 32k: M = 1 0.096 vs 0.125 ms, M = 2 0.127 vs 0.126, M = 4 0.202 vs 0.126, M = 16 0.352 vs 0.128).
+constexpr int kDecodeSimtMaxM = 1;
+constexpr int kDecodeMaxM = 128;          // one 128-row query tile on the tensor-core path
+// Tensor-core variant (M up to 128): 128-key tiles, one CTA per SM; tensor maps with 128-row
+// boxes over q ([B,M,H,D]), k and v.
+int decode_splits_tc(int B, int N, int H, int n_sm, int* tiles_per_split);
+cudaError_t launch_decode_tc_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                                   float* lse, float* part_o, float* part_ml, int B, int M, int N, int H, int S,
+                                   int tiles_per_split, int* err, cudaStream_t st);
 int decode_splits(int B, int N, int H, int n_sm, int* tiles_per_split);
 cudaError_t launch_decode_sm100(const CUtensorMap& tk, const CUtensorMap& tv, const void* q, void* o, float* lse,
                                 float* part_o, float* part_ml, int B, int M, int N, int H, int S,

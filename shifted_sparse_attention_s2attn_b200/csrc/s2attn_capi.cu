@@ -186,13 +186,11 @@ int sm_count() {
   return cache[dev];
 }
 
-constexpr int kDecodeMaxM = 16;
-
 int check_decode_shape(int B, int M, int N, int H, int D) {
   if (B < 1 || M < 1 || N < 1 || H < 1 || D < 1 || M > N) return S2ATTN_ERR_INVALID_ARG;
   if ((long long)B * N > INT_MAX / 2) return S2ATTN_ERR_INVALID_ARG;
   if ((long long)B * N * H > (LLONG_MAX / 8) / D) return S2ATTN_ERR_INVALID_ARG;
-  if (D != 128 || M > kDecodeMaxM) return S2ATTN_ERR_UNSUPPORTED;
+  if (D != 128 || M > s2::kDecodeMaxM) return S2ATTN_ERR_UNSUPPORTED;
   if ((long long)B * H * M > INT_MAX || (long long)B * H * s2::kDecodeMaxSplits > INT_MAX)
     return S2ATTN_ERR_UNSUPPORTED;
   return S2ATTN_OK;
@@ -315,18 +313,26 @@ int s2attn_decode(const void* q, const void* k, const void* v, void* o, float* l
     return S2ATTN_ERR_WORKSPACE;
   const int n_sm = sm_count();
   if (n_sm <= 0) return S2ATTN_ERR_CUDA;
-  int tps = 0;
-  const int S = s2::decode_splits(B, N, H, n_sm, &tps);
   float* part_o = static_cast<float*>(workspace);
   float* part_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_part_o_bytes(B, M, N, H, D));
   const s2::Shape s{B, N, H, D, N, 0};
-  CUtensorMap tk, tv;
-  if (!map_bf16_sw128(&tk, k, s, s2::kDecodeTileKeys) || !map_bf16_sw128(&tv, v, s, s2::kDecodeTileKeys))
-    return S2ATTN_ERR_CUDA;
   int* err = error_word_ptr();
   if (!err) return S2ATTN_ERR_CUDA;
-  return cuda_status(s2::launch_decode_sm100(tk, tv, q, o, lse, part_o, part_ml, B, M, N, H, S, tps, err,
-                                             static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int tps = 0;
+  if (M <= s2::kDecodeSimtMaxM) {
+    const int S = s2::decode_splits(B, N, H, n_sm, &tps);
+    CUtensorMap tk, tv;
+    if (!map_bf16_sw128(&tk, k, s, s2::kDecodeTileKeys) || !map_bf16_sw128(&tv, v, s, s2::kDecodeTileKeys))
+      return S2ATTN_ERR_CUDA;
+    return cuda_status(s2::launch_decode_sm100(tk, tv, q, o, lse, part_o, part_ml, B, M, N, H, S, tps, err, st));
+  }
+  const int S = s2::decode_splits_tc(B, N, H, n_sm, &tps);
+  const s2::Shape sq{B, M, H, D, M, 0};
+  CUtensorMap tq, tk, tv;
+  if (!map_bf16_sw128(&tq, q, sq, 128) || !map_bf16_sw128(&tk, k, s, 128) || !map_bf16_sw128(&tv, v, s, 128))
+    return S2ATTN_ERR_CUDA;
+  return cuda_status(s2::launch_decode_tc_sm100(tq, tk, tv, o, lse, part_o, part_ml, B, M, N, H, S, tps, err, st));
 }
 
 int s2attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int N, int H, int D,

@@ -2,14 +2,15 @@
 //
 // Inference runs ordinary full attention; S^2-Attn is a training-time device only
 // ("LongLoRA paper notes", section 3.1; model.aibase.cn, features list).  A decoding
-// step appends M (<= 16) tokens to a sequence of N positions: k, v [B,N,H,D] hold all
+// step appends M (<= 128) tokens to a sequence of N positions: k, v [B,N,H,D] hold all
 // N positions (the new ones included), q [B,M,H,D] the M new queries; query m sits at
 // position N-M+m and sees keys 0 .. N-M+m.
 //
-// With a handful of queries the step is a matrix-vector product over the whole K/V of
-// every head: 2*N*D*2 bytes per head and 4*M*D FLOPs per key, so it is bound by HBM, not
-// by arithmetic -- it runs on the CUDA cores, and its job is to stream K and V at full
-// bandwidth:
+// Two kernels, chosen by M (kDecodeSimtMaxM).  With one query the step is a matrix-vector
+// product over the whole K/V of every head: 2*N*D*2 bytes per head and 4*D FLOPs per key,
+// bound by HBM, not by arithmetic -- the first kernel runs on the CUDA cores, and its job
+// is to stream K and V at full bandwidth (it is written for up to 16 queries, but from two
+// queries on the tensor-core kernel further down is faster):
 //   * split-KV: CTA (b, h, split) takes a run of 64-key tiles of one head, so that the
 //     grid fills every SM even for one sequence (B*H*splits CTAs, sized to whole waves);
 //   * a producer thread streams the tiles with TMA (four 64-row x 64-column boxes per
@@ -407,6 +408,299 @@ cudaError_t launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const Par
 
 }  // namespace dec
 
+// ---------------------------------------------------------------------------------------
+// Tensor-core decoding step for more queries (M up to 128: speculative decoding, chunked
+// prefill).  With M > 8 the CUDA-core kernel runs out of arithmetic (4*M*D FLOPs per key),
+// so here the step is the forward's tcgen05 machinery on one query tile of 128 rows (rows
+// >= M are padding and discarded) against the split's 128-key tiles:
+//   S(i) = Q K(i)^T (SS, fp32 in TMEM, two buffers), P(i) = exp2(S*scale*log2e - m) written
+//   back over S(i) as bf16, O += P(i) V(i) (TS), online softmax with the lazy rescale.
+// The issue order S(i) | PV(i-1) lets the softmax of tile i-1 run while S(i) computes; the
+// step stays bound by HBM up to M = 128 (16 MMAs and one 128-row softmax per 64 KB tile).
+// Warps 0-3: softmax (thread = query row = TMEM lane); warp 4: TMA producer and TMEM
+// owner; warp 5: MMA issuer.  The partials go to the same workspace layout as above.
+namespace dtc {
+
+constexpr int HD = 128, BM = 128, BN = 128;
+constexpr uint32_t BOX = 128 * 128;           // 128 rows x 128 B (64 bf16 columns)
+constexpr uint32_t TILE = 2 * BOX;            // 128 rows x 128 bf16
+constexpr int NST = 3;                        // K/V ring stages
+constexpr int NTHREADS = 192;
+constexpr int WARP_LOAD = 4, WARP_MMA = 5;
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + TILE;              // [NST]
+constexpr uint32_t OFF_V = OFF_K + NST * TILE;        // [NST]
+constexpr uint32_t OFF_BAR = OFF_V + NST * TILE;
+// barriers: q_full, kv_full[NST], kv_empty[NST], s_full[2], p_ready[2], pv_done, o_final, drain.
+// p_ready is double-buffered by tile parity: S(i) is issued before the wait for P(i-1), so
+// the softmax may finish tile i before that wait looks; with a single barrier it would then
+// be two phases ahead and the parity wait would miss the completed phase.
+constexpr int NBARS = 1 + 2 * NST + 2 + 2 + 3;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
+constexpr uint32_t TM_O = 256;                          // S buffers at columns 0 and 128
+
+struct Params {
+  float* part_o;
+  float* part_ml;
+  int B, M, N, H, S, tiles_per_split;
+  float sl2;  // log2(e) / sqrt(D)
+  int* err;
+};
+
+enum Site : int { SITE_LOAD = 5, SITE_MMA = 6, SITE_SOFTMAX = 7, SITE_DRAIN = 8 };
+
+__device__ __forceinline__ void issue_s(uint32_t d, uint32_t sq, uint32_t sk, uint32_t idesc) {
+  const uint64_t dq = sdesc_sw128(sq, 16, 1024), dk = sdesc_sw128(sk, 16, 1024);
+#pragma unroll
+  for (int kk = 0; kk < HD / 16; ++kk) {
+    const uint32_t off = (kk / 4) * BOX + (kk % 4) * 32;
+    mma_ss(d, sdesc_add(dq, off), sdesc_add(dk, off), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ void issue_pv(uint32_t d, uint32_t tp, uint32_t sv, uint32_t idesc, bool first) {
+  const uint64_t dv = sdesc_sw128(sv, BOX, 1024);  // V^T viewed MN-major, 64-column boxes BOX apart
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk) mma_ts(d, tp + kk * 8, sdesc_add(dv, kk * 2048), idesc, (first && kk == 0) ? 0u : 1u);
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// P row = exp2(s * sl2 - m) with columns c > lim masked, written as bf16 pairs over the first
+// 64 TMEM columns of the row's S buffer; returns the fp32 row sum.
+__device__ __forceinline__ float p_row(const uint32_t (&s0)[64], const uint32_t (&s1)[64], int lim, float sl2,
+                                       float neg_m, uint32_t t_s) {
+  const float2 scale2 = make_float2(sl2, sl2), shift2 = make_float2(neg_m, neg_m);
+  float2 sp[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) sp[e] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const uint32_t(&sr)[64] = hh == 0 ? s0 : s1;
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, shift2);
+      float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+      p0 = 64 * hh + 2 * c <= lim ? p0 : 0.f;
+      p1 = 64 * hh + 2 * c + 1 <= lim ? p1 : 0.f;
+      sp[c % 4].x += p0;
+      sp[c % 4].y += p1;
+      pk[c] = pack_bf16x2(p0, p1);
+    }
+    tmem_st_x32(t_s + 32 * hh, pk);
+  }
+  return ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + NST;
+  uint64_t* s_full = bars + 1 + 2 * NST;  // [2]
+  uint64_t* p_ready = s_full + 2;         // [2]
+  uint64_t* pv_done = s_full + 4;
+  uint64_t* o_final = s_full + 5;
+  uint64_t* drain = s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int units = p.B * p.H;
+  const int bh = (int)(blockIdx.x % units);  // consecutive CTAs: the same split of consecutive heads
+  const int split = (int)(blockIdx.x / units);
+  const int h = bh % p.H, b = bh / p.H;
+  const int t_begin = split * p.tiles_per_split * BN;
+  const int t_end = min(p.N, t_begin + p.tiles_per_split * BN);
+  const int n_tiles = t_end > t_begin ? (t_end - t_begin + BN - 1) / BN : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(&p_ready[0], 4);
+    mbar_init(&p_ready[1], 4);
+    mbar_init(pv_done, 1);
+    mbar_init(o_final, 1);
+    mbar_init(drain, 1);
+    *abort_flag = (*(volatile int*)p.err != 0) ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_LOAD) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = *abort_flag != 0 || n_tiles == 0;
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (!skip && warp == WARP_LOAD && lane == 0) {
+    // ---------------- TMA producer ----------------
+    prefetch_tmap(&tq);
+    prefetch_tmap(&tk);
+    prefetch_tmap(&tv);
+    bool ok = true;
+    int issued = 0;
+    mbar_arrive_expect_tx(q_full, TILE);
+    for (int x = 0; x < 2; ++x) tma_load_3d(smem + OFF_Q + x * BOX, &tq, x * 64, h, b * p.M, q_full);
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const int slot = i % NST;
+      if (i >= NST) ok = wait_bounded(&kv_empty[slot], ((i / NST) - 1) & 1, abort_flag, p.err);
+      if (!ok) break;
+      const int row = b * p.N + t_begin + i * BN;
+      mbar_arrive_expect_tx(&kv_full[slot], 2 * TILE);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_3d(smem + OFF_K + slot * TILE + x * BOX, &tk, x * 64, h, row, &kv_full[slot]);
+        tma_load_3d(smem + OFF_V + slot * TILE + x * BOX, &tv, x * 64, h, row, &kv_full[slot]);
+      }
+      issued = i + 1;
+    }
+    if (!ok) {
+      report_error(p.err, (K_DEC << 8) | SITE_LOAD);
+      *abort_flag = 1;
+    }
+    bool dok = wait_drain(q_full, 0);
+    for (int i = (issued > NST ? issued - NST : 0); i < issued; ++i) dok &= wait_drain(&kv_full[i % NST], (i / NST) & 1);
+    if (!dok) report_error(p.err, (K_DEC << 8) | SITE_DRAIN);
+  } else if (!skip && warp == WARP_MMA && lane == 0) {
+    // ---------------- MMA issuer: S(i) | PV(i-1) ----------------
+    const uint32_t id_s = idesc_bf16_f32(BM, BN, false, false);
+    const uint32_t id_pv = idesc_bf16_f32(BM, HD, false, true);
+    const uint32_t sq = smem_u32(smem + OFF_Q), sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
+    bool ok = wait_bounded(q_full, 0, abort_flag, p.err);
+    for (int i = 0; i <= n_tiles && ok; ++i) {
+      if (i < n_tiles) {
+        ok = wait_bounded(&kv_full[i % NST], (i / NST) & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(tmem + 128u * (i & 1), sq, sk + (i % NST) * TILE, id_s);
+        mma_commit(&s_full[i & 1]);
+      }
+      if (i > 0) {
+        ok = wait_bounded(&p_ready[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(tmem + TM_O, tmem + 128u * ((i - 1) & 1), sv + ((i - 1) % NST) * TILE, id_pv, i == 1);
+        mma_commit(pv_done);
+        mma_commit(&kv_empty[(i - 1) % NST]);
+      }
+    }
+    if (ok) mma_commit(o_final);
+    if (!ok) {
+      report_error(p.err, (K_DEC << 8) | SITE_MMA);
+      *abort_flag = 1;
+    }
+    mma_commit(drain);
+    if (!wait_drain(drain, 0)) report_error(p.err, (K_DEC << 8) | SITE_DRAIN);
+  } else if (!skip && warp < 4) {
+    // ---------------- softmax: thread = query row r ----------------
+    const int r = warp * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const float sl2 = p.sl2;
+    const int last_vis = min(p.N - p.M + r, t_end - 1);  // last key row r sees in this split
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const int buf = i & 1;
+      ok = wait_bounded(&s_full[buf], (i >> 1) & 1, abort_flag, p.err);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t t_s = lane_addr + 128u * buf;
+      uint32_t s0[64], s1[64];
+      tmem_ld_x64(t_s, s0);
+      tmem_ld_x64(t_s + 64, s1);
+      const int lim = last_vis - (t_begin + i * BN);  // columns c <= lim are visible (may be < 0)
+      float mxp[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c)
+        mxp[c % 8] = max3f(mxp[c % 8], c <= lim ? __uint_as_float(s0[c]) : -INFINITY,
+                           c + 64 <= lim ? __uint_as_float(s1[c]) : -INFINITY);
+      const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+      // lazy rescale: move the running max only when it grows by more than 2^8 (a row that has
+      // seen no visible key yet keeps -inf, and its P stays 0)
+      const float m_new = fmaxf(m_run, mx * sl2);
+      const bool need = (m_new - m_run) > 8.0f;
+      const bool rescale = __any_sync(0xffffffffu, need);
+      const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
+      if (need) m_run = m_new;
+      l_run *= alpha;
+      l_run += p_row(s0, s1, lim, sl2, -m_run, t_s);
+      if (rescale && i > 0) {
+        // O was last written by PV(i-1): wait for it, then scale this row of O
+        ok = wait_bounded(pv_done, (i - 1) & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < HD; c += 32) {
+          uint32_t rr[32];
+          tmem_ld_x32(lane_addr + TM_O + c, rr);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+          tmem_st_x32(lane_addr + TM_O + c, rr);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_ready[buf]);
+    }
+    if (ok) ok = wait_bounded(o_final, 0, abort_flag, p.err);
+    if (ok) {
+      // partial of this split: unnormalised O row, running max (log2 domain) and sum
+      tc_fence_after();
+      const size_t part = (size_t)bh * p.S + split;
+#pragma unroll
+      for (int c = 0; c < HD; c += 32) {
+        uint32_t rr[32];
+        tmem_ld_x32(lane_addr + TM_O + c, rr);
+        if (r < p.M) {
+          float4* dst = reinterpret_cast<float4*>(p.part_o + (part * p.M + r) * HD + c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(rr[4 * e]), __uint_as_float(rr[4 * e + 1]),
+                                 __uint_as_float(rr[4 * e + 2]), __uint_as_float(rr[4 * e + 3]));
+        }
+      }
+      if (r < p.M) {
+        p.part_ml[(part * p.M + r) * 2] = m_run;
+        p.part_ml[(part * p.M + r) * 2 + 1] = l_run;
+      }
+    } else {
+      report_error(p.err, (K_DEC << 8) | SITE_SOFTMAX);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_LOAD) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace dtc
+
 int decode_splits(int B, int N, int H, int n_sm, int* tiles_per_split) {
   const int n_tiles = (N + dec::TK - 1) / dec::TK;
   const long long units = (long long)B * H;
@@ -420,6 +714,70 @@ int decode_splits(int B, int N, int H, int n_sm, int* tiles_per_split) {
   const int tps = (int)((n_tiles + s - 1) / s);
   *tiles_per_split = tps;
   return (n_tiles + tps - 1) / tps;
+}
+
+// The combine kernel is a programmatic dependent launch: it is scheduled while the split
+// kernel drains, which hides its launch latency.
+static cudaError_t launch_combine(const float* part_o, const float* part_ml, void* o, float* lse, int B, int M,
+                                  int H, int S, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((long long)B * H * M));
+  cfg.blockDim = dim3(dec::CG * dec::HD);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, dec::decode_combine_kernel, part_o, part_ml, static_cast<__nv_bfloat16*>(o), lse,
+                            M, H, S);
+}
+
+int decode_splits_tc(int B, int N, int H, int n_sm, int* tiles_per_split) {
+  const int n_tiles = (N + dtc::BN - 1) / dtc::BN;
+  const long long units = (long long)B * H;
+  const long long base_ctas = units * ((n_tiles + 7) / 8);  // about 8 tiles (1024 keys) per CTA
+  const long long waves = (base_ctas + n_sm - 1) / n_sm;     // one CTA per SM
+  long long s = (waves * n_sm) / units;
+  if (s < 1) s = 1;
+  if (s > n_tiles) s = n_tiles;
+  if (s > kDecodeMaxSplits) s = kDecodeMaxSplits;
+  const int tps = (int)((n_tiles + s - 1) / s);
+  *tiles_per_split = tps;
+  return (n_tiles + tps - 1) / tps;
+}
+
+cudaError_t launch_decode_tc_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                                   float* lse, float* part_o, float* part_ml, int B, int M, int N, int H, int S,
+                                   int tiles_per_split, int* err, cudaStream_t st) {
+  dtc::Params p;
+  p.part_o = part_o;
+  p.part_ml = part_ml;
+  p.B = B;
+  p.M = M;
+  p.N = N;
+  p.H = H;
+  p.S = S;
+  p.tiles_per_split = tiles_per_split;
+  p.sl2 = (float)(1.4426950408889634 / sqrt((double)dtc::HD));
+  p.err = err;
+  const long long grid = (long long)B * H * S;
+  if (grid <= 0 || grid > 0x7fffffffLL || M < 1 || M > dtc::BM) return cudaErrorInvalidValue;
+  static std::atomic<uint64_t> done_mask{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (!bit || !(done_mask.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(dtc::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dtc::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  dtc::decode_tc_kernel<<<(unsigned)grid, dtc::NTHREADS, dtc::SMEM_BYTES, st>>>(tq, tk, tv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_combine(part_o, part_ml, o, lse, B, M, H, S, st);
 }
 
 cudaError_t launch_decode_sm100(const CUtensorMap& tk, const CUtensorMap& tv, const void* q, void* o, float* lse,
@@ -439,27 +797,11 @@ cudaError_t launch_decode_sm100(const CUtensorMap& tk, const CUtensorMap& tv, co
   p.err = err;
   const long long grid = (long long)B * H * S;
   if (grid <= 0 || grid > 0x7fffffffLL || M < 1 || M > dec::MAXM) return cudaErrorInvalidValue;
-  cudaError_t e;
-  if (M == 1) e = dec::launch_split<1>(tk, tv, p, st);
-  else if (M == 2) e = dec::launch_split<2>(tk, tv, p, st);
-  else if (M <= 4) e = dec::launch_split<4>(tk, tv, p, st);
-  else if (M <= 8) e = dec::launch_split<8>(tk, tv, p, st);
-  else e = dec::launch_split<16>(tk, tv, p, st);
+  static_assert(kDecodeSimtMaxM == 1, "instantiate decode_split_kernel for the query counts dispatched here");
+  if (M != 1) return cudaErrorInvalidValue;
+  cudaError_t e = dec::launch_split<1>(tk, tv, p, st);
   if (e != cudaSuccess) return e;
-  // the combine kernel is a programmatic dependent launch: it is scheduled while the
-  // split kernel drains, which hides its launch latency
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((long long)B * H * M));
-  cfg.blockDim = dim3(dec::CG * dec::HD);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, dec::decode_combine_kernel, static_cast<const float*>(part_o),
-                            static_cast<const float*>(part_ml), static_cast<__nv_bfloat16*>(o), lse, M, H, S);
+  return launch_combine(part_o, part_ml, o, lse, B, M, H, S, st);
 }
 
 }  // namespace s2

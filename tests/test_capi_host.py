@@ -92,7 +92,7 @@ def test_rope_validation(lib):
     ((1, 0, 100, 2, 128), -1),     # no query
     ((1, 5, 4, 2, 128), -1),       # more queries than positions
     ((0, 1, 100, 2, 128), -1),     # empty batch
-    ((1, 17, 100, 2, 128), -2),    # more than 16 queries
+    ((1, 129, 200, 2, 128), -2),   # more than 128 queries
     ((1, 1, 100, 2, 64), -2),      # D = 64
     ((1, 1, 100, 2, 128), -1),     # valid shape, null pointers
 ])

@@ -1,5 +1,6 @@
 """GPU parity of the decoding step (full causal attention of the last M positions)
-against the fp64 oracle, through the C ABI.
+against the fp64 oracle, through the C ABI: the CUDA-core kernel (M = 1) and the
+tensor-core kernel (2 <= M <= 128).
 
 Inference runs ordinary full attention ("LongLoRA paper notes", section 3.1): the
 decoding queries are the last M positions of a sequence whose K/V hold all N
@@ -55,11 +56,20 @@ def _check(o, lse, ref_o, ref_lse):
 @pytest.mark.parametrize("B,M,N,H", [
     (1, 1, 1, 1),        # one position: o = v
     (1, 1, 128, 2),      # exactly one tile
-    (2, 3, 1000, 4),     # ragged tail, several splits, M padded to 4
-    (1, 5, 4099, 3),     # M padded to 8, tail of 3 keys
-    (1, 16, 300, 2),     # largest M, M > the last tile's tail
+    (1, 1, 20000, 2),    # many tiles per split
+    (3, 1, 777, 5),
+    # tensor-core path (2 <= M <= 128)
+    (2, 3, 1000, 4),     # ragged tail, several splits
+    (1, 5, 4099, 3),     # tail of 3 keys
+    (1, 16, 300, 2),     # M > the last tile's tail
     (1, 2, 20000, 2),    # many tiles per split
     (3, 8, 777, 5),
+    (1, 17, 300, 2),     # the last split starts past some queries' limits
+    (2, 32, 1000, 3),
+    (1, 64, 4099, 2),
+    (1, 100, 100, 2),    # M = N: the first query sees one key
+    (1, 128, 2048, 2),   # a whole query tile
+    (3, 40, 777, 5),
 ])
 def test_decode_matches_oracle(B, M, N, H):
     D = 128
@@ -92,7 +102,7 @@ def test_decode_repeated_calls_and_nonfinite_free():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)  # no atomics: the result is deterministic
 
 
-@pytest.mark.parametrize("M", [1, 16])
+@pytest.mark.parametrize("M", [1, 16, 128])
 def test_decode_llama2_7b_32k_full_size(M):
     """The 32k LLaMA2-7B layer (H=32, D=128): the decoding queries are the last M rows of
     the workload's Q, against the workload's whole K and V."""
@@ -102,3 +112,24 @@ def test_decode_llama2_7b_32k_full_size(M):
     o, lse = _run(q, k, v)
     ref_o, ref_lse = oracle.decode(q, k, v)
     _check(o, lse, ref_o, ref_lse)
+
+
+@pytest.mark.parametrize("M", [1, 16, 128])
+def test_decode_back_to_back_calls(M):
+    """Thirty calls queued back to back (no synchronisation in between, so kernels of one
+    call overlap the launches of the next): no bounded wait may give up (the device error
+    word stays clear) and the result equals a single synchronised call's."""
+    B, N, H, D = 1, 8192, 8, 128
+    q, k, v = (bits_to_device(_bits(s, 40 + i)) for i, s in enumerate([(B, M, H, D), (B, N, H, D), (B, N, H, D)]))
+    o_ref = torch.empty_like(q)
+    lse_ref = torch.empty((B, H, M), dtype=torch.float32, device="cuda")
+    ws = torch.empty(s2.s2attn_decode_workspace_bytes(B, M, N, H, D), dtype=torch.uint8, device="cuda")
+    s2.s2attn_decode(q, k, v, o_ref, lse_ref, ws)
+    torch.cuda.synchronize()
+    o, lse = torch.empty_like(o_ref), torch.empty_like(lse_ref)
+    for _ in range(30):
+        s2.s2attn_decode(q, k, v, o, lse, ws)
+    torch.cuda.synchronize()
+    rc, detail = s2.get_device_error()
+    assert rc == 0, f"device error word set: {detail:#x}"
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)

@@ -104,6 +104,7 @@ SMALL = {
     "full_causal": (1, 1024, 2, 1024, 0, 0.25),
     "one_tile_groups": (1, 512, 2, 128, 0, None),
     "all_heads_shifted": (1, 512, 2, 256, 2, None),
+    "one_group_shifted": (1, 512, 2, 512, 1, None),   # G = N with a shifted head: causal in half-rolled order
 }
 
 
