@@ -54,8 +54,8 @@ constexpr int kDecodeTileKeys = 64;       // key tile of the CUDA-core kernel (i
 // 32k: M = 1 0.096 vs 0.125 ms, M = 2 0.127 vs 0.126, M = 4 0.202 vs 0.126, M = 16 0.352 vs 0.128).
 constexpr int kDecodeSimtMaxM = 1;
 constexpr int kDecodeMaxM = 128;          // one 128-row query tile on the tensor-core path
-// Tensor-core variant (M up to 128): 128-key tiles, one CTA per SM; tensor maps with 128-row
-// boxes over q ([B,M,H,D]), k and v.
+// Tensor-core variant (M up to 128): 64-key tiles, two CTAs per SM; tensor maps with 128-row
+// boxes over q ([B,M,H,D]) and kDecodeTileKeys-row boxes over k and v.
 int decode_splits_tc(int B, int N, int H, int n_sm, int* tiles_per_split);
 cudaError_t launch_decode_tc_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                                    float* lse, float* part_o, float* part_ml, int B, int M, int N, int H, int S,

@@ -330,7 +330,8 @@ int s2attn_decode(const void* q, const void* k, const void* v, void* o, float* l
   const int S = s2::decode_splits_tc(B, N, H, n_sm, &tps);
   const s2::Shape sq{B, M, H, D, M, 0};
   CUtensorMap tq, tk, tv;
-  if (!map_bf16_sw128(&tq, q, sq, 128) || !map_bf16_sw128(&tk, k, s, 128) || !map_bf16_sw128(&tv, v, s, 128))
+  if (!map_bf16_sw128(&tq, q, sq, 128) || !map_bf16_sw128(&tk, k, s, s2::kDecodeTileKeys) ||
+      !map_bf16_sw128(&tv, v, s, s2::kDecodeTileKeys))
     return S2ATTN_ERR_CUDA;
   return cuda_status(s2::launch_decode_tc_sm100(tq, tk, tv, o, lse, part_o, part_ml, B, M, N, H, S, tps, err, st));
 }

@@ -412,25 +412,29 @@ cudaError_t launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const Par
 // Tensor-core decoding step for more queries (M up to 128: speculative decoding, chunked
 // prefill).  With M > 8 the CUDA-core kernel runs out of arithmetic (4*M*D FLOPs per key),
 // so here the step is the forward's tcgen05 machinery on one query tile of 128 rows (rows
-// >= M are padding and discarded) against the split's 128-key tiles:
-//   S(i) = Q K(i)^T (SS, fp32 in TMEM, two buffers), P(i) = exp2(S*scale*log2e - m) written
-//   back over S(i) as bf16, O += P(i) V(i) (TS), online softmax with the lazy rescale.
-// The issue order S(i) | PV(i-1) lets the softmax of tile i-1 run while S(i) computes; the
-// step stays bound by HBM up to M = 128 (16 MMAs and one 128-row softmax per 64 KB tile).
-// Warps 0-3: softmax (thread = query row = TMEM lane); warp 4: TMA producer and TMEM
-// owner; warp 5: MMA issuer.  The partials go to the same workspace layout as above.
+// >= M are padding and discarded) against the split's 64-key tiles:
+//   S(i) = Q K(i)^T (SS, N = 64, fp32 in TMEM, two buffers), P(i) = exp2(S*scale*log2e - m)
+//   written back over S(i) as bf16, O += P(i) V(i) (TS), online softmax with the lazy rescale.
+// The issue order S(i) | PV(i-1) lets the softmax of tile i-1 run while S(i) computes.
+// 64-key tiles keep a CTA at 256 TMEM columns and ~97 KB of shared memory, so two CTAs share
+// an SM and one's start-up (TMEM allocation, the Q tile, the first K/V latency) overlaps the
+// other's streaming.  Warps 0-3: softmax (thread = query row = TMEM lane); warp 4: TMA
+// producer and TMEM owner; warp 5: MMA issuer.  The partials go to the same workspace
+// layout as above.
 namespace dtc {
 
-constexpr int HD = 128, BM = 128, BN = 128;
-constexpr uint32_t BOX = 128 * 128;           // 128 rows x 128 B (64 bf16 columns)
-constexpr uint32_t TILE = 2 * BOX;            // 128 rows x 128 bf16
-constexpr int NST = 3;                        // K/V ring stages
+constexpr int HD = 128, BM = 128, BN = kDecodeTileKeys;  // 64 keys per tile
+constexpr uint32_t QBOX = BM * 128;           // 128 rows x 128 B (64 bf16 columns)
+constexpr uint32_t KBOX = BN * 128;           // 64 rows x 128 B
+constexpr uint32_t QTILE = 2 * QBOX;          // 128 query rows x 128 bf16
+constexpr uint32_t KTILE = 2 * KBOX;          // 64 key rows x 128 bf16
+constexpr int NST = 2;                        // K/V ring stages
 constexpr int NTHREADS = 192;
 constexpr int WARP_LOAD = 4, WARP_MMA = 5;
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + TILE;              // [NST]
-constexpr uint32_t OFF_V = OFF_K + NST * TILE;        // [NST]
-constexpr uint32_t OFF_BAR = OFF_V + NST * TILE;
+constexpr uint32_t OFF_K = OFF_Q + QTILE;             // [NST]
+constexpr uint32_t OFF_V = OFF_K + NST * KTILE;       // [NST]
+constexpr uint32_t OFF_BAR = OFF_V + NST * KTILE;
 // barriers: q_full, kv_full[NST], kv_empty[NST], s_full[2], p_ready[2], pv_done, o_final, drain.
 // p_ready is double-buffered by tile parity: S(i) is issued before the wait for P(i-1), so
 // the softmax may finish tile i before that wait looks; with a single barrier it would then
@@ -438,7 +442,9 @@ constexpr uint32_t OFF_BAR = OFF_V + NST * TILE;
 constexpr int NBARS = 1 + 2 * NST + 2 + 2 + 3;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1024 B
-constexpr uint32_t TM_O = 256;                          // S buffers at columns 0 and 128
+static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs must fit on an SM");
+constexpr uint32_t TM_COLS = 256;                       // two CTAs per SM
+constexpr uint32_t TM_O = 128;                          // S buffers at columns 0 and 64
 
 struct Params {
   float* part_o;
@@ -450,17 +456,20 @@ struct Params {
 
 enum Site : int { SITE_LOAD = 5, SITE_MMA = 6, SITE_SOFTMAX = 7, SITE_DRAIN = 8 };
 
+// S[128 x 64] = Q K^T: both K-major; the 64-column halves of the head dim are QBOX / KBOX apart.
 __device__ __forceinline__ void issue_s(uint32_t d, uint32_t sq, uint32_t sk, uint32_t idesc) {
   const uint64_t dq = sdesc_sw128(sq, 16, 1024), dk = sdesc_sw128(sk, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < HD / 16; ++kk) {
-    const uint32_t off = (kk / 4) * BOX + (kk % 4) * 32;
-    mma_ss(d, sdesc_add(dq, off), sdesc_add(dk, off), idesc, kk > 0 ? 1u : 0u);
+    mma_ss(d, sdesc_add(dq, (kk / 4) * QBOX + (kk % 4) * 32), sdesc_add(dk, (kk / 4) * KBOX + (kk % 4) * 32), idesc,
+           kk > 0 ? 1u : 0u);
   }
 }
 
+// O[128 x 128] += P V: P (bf16 pairs) from TMEM, V^T viewed MN-major (64-dim blocks KBOX apart,
+// 16 key rows = 2 KB per k-step).
 __device__ __forceinline__ void issue_pv(uint32_t d, uint32_t tp, uint32_t sv, uint32_t idesc, bool first) {
-  const uint64_t dv = sdesc_sw128(sv, BOX, 1024);  // V^T viewed MN-major, 64-column boxes BOX apart
+  const uint64_t dv = sdesc_sw128(sv, KBOX, 1024);
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) mma_ts(d, tp + kk * 8, sdesc_add(dv, kk * 2048), idesc, (first && kk == 0) ? 0u : 1u);
 }
@@ -472,33 +481,28 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 }
 
 // P row = exp2(s * sl2 - m) with columns c > lim masked, written as bf16 pairs over the first
-// 64 TMEM columns of the row's S buffer; returns the fp32 row sum.
-__device__ __forceinline__ float p_row(const uint32_t (&s0)[64], const uint32_t (&s1)[64], int lim, float sl2,
-                                       float neg_m, uint32_t t_s) {
+// 32 TMEM columns of the row's S buffer; returns the fp32 row sum.
+__device__ __forceinline__ float p_row(const uint32_t (&sr)[64], int lim, float sl2, float neg_m, uint32_t t_s) {
   const float2 scale2 = make_float2(sl2, sl2), shift2 = make_float2(neg_m, neg_m);
   float2 sp[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) sp[e] = make_float2(0.f, 0.f);
+  uint32_t pk[32];
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const uint32_t(&sr)[64] = hh == 0 ? s0 : s1;
-    uint32_t pk[32];
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, shift2);
-      float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-      p0 = 64 * hh + 2 * c <= lim ? p0 : 0.f;
-      p1 = 64 * hh + 2 * c + 1 <= lim ? p1 : 0.f;
-      sp[c % 4].x += p0;
-      sp[c % 4].y += p1;
-      pk[c] = pack_bf16x2(p0, p1);
-    }
-    tmem_st_x32(t_s + 32 * hh, pk);
+  for (int c = 0; c < 32; ++c) {
+    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, shift2);
+    float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+    p0 = 2 * c <= lim ? p0 : 0.f;
+    p1 = 2 * c + 1 <= lim ? p1 : 0.f;
+    sp[c % 4].x += p0;
+    sp[c % 4].y += p1;
+    pk[c] = pack_bf16x2(p0, p1);
   }
+  tmem_st_x32(t_s, pk);
   return ((sp[0].x + sp[1].x) + (sp[2].x + sp[3].x)) + ((sp[0].y + sp[1].y) + (sp[2].y + sp[3].y));
 }
 
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(NTHREADS, 2)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -541,7 +545,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     fence_mbar_init();
   }
   if (warp == WARP_LOAD) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, TM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -558,17 +562,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tv);
     bool ok = true;
     int issued = 0;
-    mbar_arrive_expect_tx(q_full, TILE);
-    for (int x = 0; x < 2; ++x) tma_load_3d(smem + OFF_Q + x * BOX, &tq, x * 64, h, b * p.M, q_full);
+    mbar_arrive_expect_tx(q_full, QTILE);
+    for (int x = 0; x < 2; ++x) tma_load_3d(smem + OFF_Q + x * QBOX, &tq, x * 64, h, b * p.M, q_full);
     for (int i = 0; i < n_tiles && ok; ++i) {
       const int slot = i % NST;
       if (i >= NST) ok = wait_bounded(&kv_empty[slot], ((i / NST) - 1) & 1, abort_flag, p.err);
       if (!ok) break;
       const int row = b * p.N + t_begin + i * BN;
-      mbar_arrive_expect_tx(&kv_full[slot], 2 * TILE);
+      mbar_arrive_expect_tx(&kv_full[slot], 2 * KTILE);
       for (int x = 0; x < 2; ++x) {
-        tma_load_3d(smem + OFF_K + slot * TILE + x * BOX, &tk, x * 64, h, row, &kv_full[slot]);
-        tma_load_3d(smem + OFF_V + slot * TILE + x * BOX, &tv, x * 64, h, row, &kv_full[slot]);
+        tma_load_3d(smem + OFF_K + slot * KTILE + x * KBOX, &tk, x * 64, h, row, &kv_full[slot]);
+        tma_load_3d(smem + OFF_V + slot * KTILE + x * KBOX, &tv, x * 64, h, row, &kv_full[slot]);
       }
       issued = i + 1;
     }
@@ -590,14 +594,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ok = wait_bounded(&kv_full[i % NST], (i / NST) & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
-        issue_s(tmem + 128u * (i & 1), sq, sk + (i % NST) * TILE, id_s);
+        issue_s(tmem + (uint32_t)BN * (i & 1), sq, sk + (i % NST) * KTILE, id_s);
         mma_commit(&s_full[i & 1]);
       }
       if (i > 0) {
         ok = wait_bounded(&p_ready[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(tmem + TM_O, tmem + 128u * ((i - 1) & 1), sv + ((i - 1) % NST) * TILE, id_pv, i == 1);
+        issue_pv(tmem + TM_O, tmem + (uint32_t)BN * ((i - 1) & 1), sv + ((i - 1) % NST) * KTILE, id_pv, i == 1);
         mma_commit(pv_done);
         mma_commit(&kv_empty[(i - 1) % NST]);
       }
@@ -622,18 +626,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ok = wait_bounded(&s_full[buf], (i >> 1) & 1, abort_flag, p.err);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t t_s = lane_addr + 128u * buf;
-      uint32_t s0[64], s1[64];
+      const uint32_t t_s = lane_addr + (uint32_t)BN * buf;
+      uint32_t s0[64];
       tmem_ld_x64(t_s, s0);
-      tmem_ld_x64(t_s + 64, s1);
       const int lim = last_vis - (t_begin + i * BN);  // columns c <= lim are visible (may be < 0)
       float mxp[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 64; ++c)
-        mxp[c % 8] = max3f(mxp[c % 8], c <= lim ? __uint_as_float(s0[c]) : -INFINITY,
-                           c + 64 <= lim ? __uint_as_float(s1[c]) : -INFINITY);
+      for (int c = 0; c < 32; ++c)
+        mxp[c % 8] = max3f(mxp[c % 8], 2 * c <= lim ? __uint_as_float(s0[2 * c]) : -INFINITY,
+                           2 * c + 1 <= lim ? __uint_as_float(s0[2 * c + 1]) : -INFINITY);
       const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
                              fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
       // lazy rescale: move the running max only when it grows by more than 2^8 (a row that has
@@ -644,7 +647,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
       if (need) m_run = m_new;
       l_run *= alpha;
-      l_run += p_row(s0, s1, lim, sl2, -m_run, t_s);
+      l_run += p_row(s0, lim, sl2, -m_run, t_s);
       if (rescale && i > 0) {
         // O was last written by PV(i-1): wait for it, then scale this row of O
         ok = wait_bounded(pv_done, (i - 1) & 1, abort_flag, p.err);
@@ -695,7 +698,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   if (warp == WARP_LOAD) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, TM_COLS);
   }
 }
 
@@ -737,9 +740,10 @@ static cudaError_t launch_combine(const float* part_o, const float* part_ml, voi
 int decode_splits_tc(int B, int N, int H, int n_sm, int* tiles_per_split) {
   const int n_tiles = (N + dtc::BN - 1) / dtc::BN;
   const long long units = (long long)B * H;
-  const long long base_ctas = units * ((n_tiles + 7) / 8);  // about 8 tiles (1024 keys) per CTA
-  const long long waves = (base_ctas + n_sm - 1) / n_sm;     // one CTA per SM
-  long long s = (waves * n_sm) / units;
+  const long long slots = 2LL * n_sm;                          // two CTAs per SM
+  const long long base_ctas = units * ((n_tiles + 15) / 16);  // about 16 tiles (1024 keys) per CTA
+  const long long waves = (base_ctas + slots - 1) / slots;
+  long long s = (waves * slots) / units;
   if (s < 1) s = 1;
   if (s > n_tiles) s = n_tiles;
   if (s > kDecodeMaxSplits) s = kDecodeMaxSplits;
