@@ -114,8 +114,11 @@ int s2attn_bwd_dq_convert(const float* dq_acc, void* dq, int B, int N, int H, in
  * 128-row query tile on the tensor cores (speculative decoding, chunked prefill).
  * `workspace` (device, caller-owned, 256-byte aligned, at least
  * s2attn_decode_workspace_bytes bytes) receives per-split partial results and is
- * overwritten.  V rows past a query's causal limit are multiplied by a zero weight,
- * so k and v must hold finite values at every position.  Runs two kernels on `stream`.
+ * overwritten; its size holds fp32 partials (D outputs, max, sum per query) of at most
+ * min(64, ceil(N/64)) splits per (b, h), independent of the device; 0 means invalid sizes.
+ * V rows past a query's causal limit are multiplied by a zero weight, so k and v must hold
+ * finite values at every position.  Runs two kernels on `stream`; the second (the split
+ * combine) is a programmatic dependent launch that waits on the device for the first.
  */
 size_t s2attn_decode_workspace_bytes(int B, int M, int N, int H, int D);
 int s2attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int M, int N, int H,
