@@ -41,6 +41,8 @@ def _load():
         lib.oracle_rope_pi_f64.restype = None
         lib.oracle_rope_pi_f32_bf16.argtypes = [vp, vp, i, i, i, i, ctypes.c_float, ctypes.c_float]
         lib.oracle_rope_pi_f32_bf16.restype = None
+        lib.oracle_rope_pi_f32_bf16_at.argtypes = [vp, vp, i, i, i, i, i, ctypes.c_float, ctypes.c_float]
+        lib.oracle_rope_pi_f32_bf16_at.restype = None
         _lib = lib
     return _lib
 
@@ -153,3 +155,15 @@ def rope_pi_bf16(x_bits, pos_scale, base=10000.0):
     B, N, H, D = x.shape
     _load().oracle_rope_pi_f32_bf16(_ptr(x), _ptr(y), B, N, H, D, float(pos_scale), float(base))
     return y
+
+
+def rope_pi_bf16_at(x_bits, pos0, pos_scale, base=10000.0):
+    """As rope_pi_bf16, for a tensor whose row t is the token at position pos0 + t."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    y = np.empty_like(x)
+    B, N, H, D = x.shape
+    if pos0 < 0:
+        raise ValueError("pos0 must be >= 0")
+    _load().oracle_rope_pi_f32_bf16_at(_ptr(x), _ptr(y), B, N, H, D, int(pos0), float(pos_scale), float(base))
+    return y
+

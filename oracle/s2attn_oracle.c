@@ -393,13 +393,23 @@ static float bf16_to_f32(uint16_t h) {
  * then rounded to bf16 (nearest-even).  x and y are bf16 bit patterns [B,N,H,D];
  * in-place (x == y) is allowed.
  */
+void oracle_rope_pi_f32_bf16_at(const uint16_t *x, uint16_t *y, int B, int N, int H, int D, int pos0,
+                                float pos_scale, float base);
+
 void oracle_rope_pi_f32_bf16(const uint16_t *x, uint16_t *y, int B, int N, int H, int D,
                              float pos_scale, float base) {
+  oracle_rope_pi_f32_bf16_at(x, y, B, N, H, D, 0, pos_scale, base);
+}
+
+/* The same, for a tensor whose row t holds the token at position pos0 + t (the new tokens
+ * of a decoding step): the position index is pos0 + t, everything else as above. */
+void oracle_rope_pi_f32_bf16_at(const uint16_t *x, uint16_t *y, int B, int N, int H, int D, int pos0,
+                                float pos_scale, float base) {
   int half = D / 2;
 #pragma omp parallel for collapse(2)
   for (int b = 0; b < B; ++b)
     for (int t = 0; t < N; ++t) {
-      float pos = (float)t * pos_scale;
+      float pos = (float)(pos0 + t) * pos_scale;
       for (int i = 0; i < half; ++i) {
         float theta = (float)pow((double)base, -2.0 * (double)i / (double)D);
         float a = pos * theta;

@@ -283,3 +283,17 @@ def test_rope_bf16_commutes_with_power_of_two_scaling():
     a = oracle.rope_pi_bf16(times8(bits), 1 / 25)
     b = times8(oracle.rope_pi_bf16(bits, 1 / 25))
     np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("pos0,scale", [(0, 0.5), (7, 1.0), (4093, 0.125), (32760, 1 / 8)])
+def test_rope_at_offset_equals_rows_of_the_longer_sequence(pos0, scale):
+    """Rotating rows t of a short tensor as tokens pos0 + t (a decoding step's new rows) gives
+    exactly rows pos0 .. pos0+N-1 of the same rows rotated as part of the whole sequence."""
+    from shifted_sparse_attention_s2attn_b200.synthetic import f32_to_bf16_bits
+    B, N, H, D = 1, 5, 2, 64
+    rows = f32_to_bf16_bits(_rand((B, N, H, D), 31).astype(np.float32))
+    full = np.zeros((B, pos0 + N, H, D), dtype=np.uint16)
+    full[:, pos0:] = rows
+    np.testing.assert_array_equal(oracle.rope_pi_bf16_at(rows, pos0, scale), oracle.rope_pi_bf16(full, scale)[:, pos0:])
+    if pos0 == 0:
+        np.testing.assert_array_equal(oracle.rope_pi_bf16_at(rows, 0, scale), oracle.rope_pi_bf16(rows, scale))
