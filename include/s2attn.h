@@ -152,6 +152,18 @@ int s2attn_bwd_f32(const float* q, const float* k, const float* v, const float* 
 int rope_pi_apply(void* q, void* k, int B, int N, int H, int D, float pos_scale, float base, void* stream);
 
 /*
+ * RoPE-PI as above for tensors whose row t is the token at position pos0 + t: the new
+ * tokens of a decoding step (q and the k rows appended to the cache sit at positions
+ * N_cache - M .. N_cache - 1).  Identical, bit for bit, to rows pos0 .. pos0+N-1 of
+ * rope_pi_apply over the whole sequence (same operation order and table entries).
+ * Requires pos0 >= 0 and pos0 + N <= 2^24.  The table is built on the host and cached in
+ * device memory for the next power of two >= pos0 + N positions (at least 1024): D*4 bytes
+ * per position, 64 MB for 128k positions at D = 128.
+ */
+int rope_pi_apply_offset(void* q, void* k, int B, int N, int H, int D, int pos0, float pos_scale, float base,
+                         void* stream);
+
+/*
  * Backward pass that allocates nothing.  The LongLoRA pages have no counterpart of
  * this entry point; it exists for callers that cannot allocate device memory on
  * the call path (a runtime whose allocator already holds the device's memory, a

@@ -12,7 +12,7 @@ import os
 __all__ = [
     "S2AttnError", "capi", "library_path",
     "s2attn_fwd", "s2attn_bwd", "s2attn_bwd_workspace_bytes", "s2attn_bwd_preprocess", "s2attn_bwd_main",
-    "s2attn_bwd_dq_convert", "s2attn_bwd_noalloc", "s2attn_decode", "s2attn_decode_workspace_bytes", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply",
+    "s2attn_bwd_dq_convert", "s2attn_bwd_noalloc", "s2attn_decode", "s2attn_decode_workspace_bytes", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply", "rope_pi_apply_offset",
     "get_device_error", "clear_device_error", "s2attn_selftest_bounded_wait",
 ]
 
@@ -57,6 +57,7 @@ def capi():
         "s2attn_fwd_f32": ([P, P, P, P, P, I, I, I, I, I, I, P], I),
         "s2attn_bwd_f32": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, Z, P], I),
         "rope_pi_apply": ([P, P, I, I, I, I, F, F, P], I),
+        "rope_pi_apply_offset": ([P, P, I, I, I, I, I, F, F, P], I),
         "s2attn_get_device_error": ([ctypes.POINTER(I)], I),
         "s2attn_clear_device_error": ([], I),
         "s2attn_selftest_bounded_wait": ([ctypes.c_uint, P], I),
@@ -177,6 +178,14 @@ def rope_pi_apply(q, k, pos_scale, base=10000.0, stream=None):
     B, N, H, D = _bnhd(ref, "q/k")
     _check("rope_pi_apply", capi().rope_pi_apply(_ptr(q), _ptr(k), B, N, H, D, float(pos_scale), float(base),
                                                  _stream(stream)))
+
+
+def rope_pi_apply_offset(q, k, pos0, pos_scale, base=10000.0, stream=None):
+    """In-place RoPE-PI on bf16 q and/or k whose row t is the token at position pos0 + t."""
+    ref = q if q is not None else k
+    B, N, H, D = _bnhd(ref, "q/k")
+    _check("rope_pi_apply_offset", capi().rope_pi_apply_offset(_ptr(q), _ptr(k), B, N, H, D, int(pos0),
+                                                               float(pos_scale), float(base), _stream(stream)))
 
 
 def get_device_error():

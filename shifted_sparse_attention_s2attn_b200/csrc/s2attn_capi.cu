@@ -380,6 +380,29 @@ int rope_pi_apply(void* q, void* k, int B, int N, int H, int D, float pos_scale,
       s2::launch_rope_pi(q, k, tab.cos_d, tab.sin_d, B, N, H, D, static_cast<cudaStream_t>(stream)));
 }
 
+int rope_pi_apply_offset(void* q, void* k, int B, int N, int H, int D, int pos0, float pos_scale, float base,
+                         void* stream) {
+  if (B < 1 || N < 1 || H < 1 || D < 16 || D % 16 != 0 || D > 256 || pos0 < 0) return S2ATTN_ERR_INVALID_ARG;
+  if ((long long)pos0 + N > (1LL << 24)) return S2ATTN_ERR_INVALID_ARG;
+  if ((long long)B * N * H > (LLONG_MAX / 8) / D) return S2ATTN_ERR_INVALID_ARG;
+  if (!q && !k) return S2ATTN_ERR_INVALID_ARG;
+  if ((q && !aligned16(q)) || (k && !aligned16(k))) return S2ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(pos_scale) || !std::isfinite(base) || !(base > 0.f)) return S2ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return S2ATTN_ERR_CUDA;
+  // Row p of a table holds position p whatever the table's length, so the table of the
+  // next power of two >= pos0 + N (cached like any other) serves every offset below it,
+  // and a decoding loop that grows its sequence builds only a few tables.
+  int rows = 1024;
+  while (rows < pos0 + N) rows *= 2;
+  RopeTable tab;
+  int rc = rope_table(dev, rows, D, pos_scale, base, &tab);
+  if (rc) return rc;
+  const size_t off = (size_t)pos0 * (D / 2);
+  return cuda_status(s2::launch_rope_pi(q, k, tab.cos_d + off, tab.sin_d + off, B, N, H, D,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 int s2attn_selftest_bounded_wait(unsigned timeout_us, void* stream) {
   if (timeout_us == 0 || timeout_us > 1000000u) return S2ATTN_ERR_INVALID_ARG;
   int* err = error_word_ptr();

@@ -81,6 +81,13 @@ def test_f32_validation(lib):
     assert lib.s2attn_fwd_f32(NULL, NULL, NULL, NULL, NULL, 1, 90, 3, 256, 18, 1, NULL) == -2  # D > 128
 
 
+def test_rope_offset_validation(lib):
+    p = ctypes.c_void_p(0x1000)
+    assert lib.rope_pi_apply_offset(p, NULL, 1, 16, 2, 128, -1, 0.5, 10000.0, NULL) == -1        # negative offset
+    assert lib.rope_pi_apply_offset(p, NULL, 1, 16, 2, 128, 1 << 24, 0.5, 10000.0, NULL) == -1   # past 2^24
+    assert lib.rope_pi_apply_offset(NULL, NULL, 1, 16, 2, 128, 5, 0.5, 10000.0, NULL) == -1      # neither q nor k
+
+
 def test_rope_validation(lib):
     assert lib.rope_pi_apply(NULL, NULL, 1, 16, 2, 128, 0.5, 10000.0, NULL) == -1   # neither q nor k
     p = ctypes.c_void_p(0x1000)

@@ -210,3 +210,21 @@ def test_bf16_full_size_sampled(wname):
     if bwd:
         for g in ("dq", "dk", "dv"):
             assert torch.isfinite(out[g]).all(), g
+
+
+@pytest.mark.parametrize("pos0,N,H,D,scale", [(0, 64, 2, 128, 0.5), (4090, 16, 32, 128, 1 / 8),
+                                               (32752, 16, 32, 128, 1 / 8), (1000, 33, 3, 64, 1.0)])
+def test_rope_pi_offset_bit_exact(pos0, N, H, D, scale):
+    """Rows at positions pos0 .. pos0+N-1 (a decoding step's new tokens): bit-exact to the
+    oracle and to the same rows of rope_pi_apply over the whole sequence."""
+    from parity_utils import bits_to_device
+    q_bits, k_bits = _bits((1, N, H, D), 50), _bits((1, N, H, D), 51)
+    q, k = bits_to_device(q_bits), bits_to_device(k_bits)
+    s2.rope_pi_apply_offset(q, k, pos0, scale)
+    full = torch.zeros((1, pos0 + N, H, D), dtype=torch.bfloat16, device="cuda")
+    full[:, pos0:] = bits_to_device(q_bits)
+    s2.rope_pi_apply(full, None, scale)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(device_to_bits(q), oracle.rope_pi_bf16_at(q_bits, pos0, scale))
+    np.testing.assert_array_equal(device_to_bits(k), oracle.rope_pi_bf16_at(k_bits, pos0, scale))
+    np.testing.assert_array_equal(device_to_bits(q), device_to_bits(full[:, pos0:]))
