@@ -1,0 +1,107 @@
+"""Sequence-sharded S^2-Attn on CPU: gloo ranks exchange the G/2 halos of the shifted heads,
+run the per-rank attention (here the fp64 oracle, with shift_heads = 0 on the local
+layout), and the rows they return, put side by side, must equal the oracle on the whole
+sequence with the shift -- forward (o, lse) and backward (dq, dk, dv)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+B, N, H, D, G, SH = 2, 64, 3, 4, 8, 2
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _inputs():
+    rng = np.random.default_rng(77)
+    return [rng.standard_normal((B, N, H, D)) for _ in range(4)]
+
+
+def _oracle_fwd(q, k, v, G):
+    import oracle
+    o, lse = oracle.s2attn_fwd(q.numpy(), k.numpy(), v.numpy(), G, 0)
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def _oracle_bwd(q, k, v, o, dout, lse, G):
+    import oracle
+    # the o and lse handed over must be those of the local layout (they travel through the halo exchange)
+    o_ref, lse_ref = oracle.s2attn_fwd(q.numpy(), k.numpy(), v.numpy(), G, 0)
+    assert np.abs(o.numpy() - o_ref).max() < 1e-12 and np.abs(lse.numpy() - lse_ref).max() < 1e-12
+    dq, dk, dv = oracle.s2attn_bwd(q.numpy(), k.numpy(), v.numpy(), dout.numpy(), G, 0)
+    return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv)
+
+
+def _run_rank(rank, world):
+    import sys
+    sys.path.insert(0, ROOT)
+    from shifted_sparse_attention_s2attn_b200.sharded import shard_range, sharded_bwd, sharded_fwd
+    t0, t1 = shard_range(N, G, world, rank)
+    q, k, v, do = (torch.from_numpy(x[:, t0:t1].copy()) for x in _inputs())
+    o, lse = sharded_fwd(q, k, v, G, SH, attn_fwd=_oracle_fwd)
+    dq, dk, dv = sharded_bwd(q, k, v, o, do, lse, G, SH, attn_bwd=_oracle_bwd)
+    return [x.numpy() for x in (o, lse, dq, dk, dv)]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    from datetime import timedelta
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=timedelta(seconds=60))
+    try:
+        q.put((rank, _run_rank(rank, world)))
+    finally:
+        dist.destroy_process_group()
+
+
+def _check(parts):
+    import sys
+    sys.path.insert(0, ROOT)
+    import oracle
+    o = np.concatenate([p[0] for p in parts], axis=1)
+    lse = np.concatenate([p[1] for p in parts], axis=2)
+    dq, dk, dv = (np.concatenate([p[i] for p in parts], axis=1) for i in (2, 3, 4))
+    qf, kf, vf, dof = _inputs()
+    ro, rlse = oracle.s2attn_fwd(qf, kf, vf, G, SH)
+    rdq, rdk, rdv = oracle.s2attn_bwd(qf, kf, vf, dof, G, SH)
+    for got, ref in ((o, ro), (lse, rlse), (dq, rdq), (dk, rdk), (dv, rdv)):
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_one_rank_wraps_onto_itself():
+    _check([_run_rank(0, 1)])
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_match_the_unsharded_oracle(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    try:
+        results = dict(q.get(timeout=120) for _ in range(world))
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+    assert all(p.exitcode == 0 for p in procs)
+    _check([results[r] for r in range(world)])
+
+
+def test_shard_range_rejects_partial_groups():
+    from shifted_sparse_attention_s2attn_b200.sharded import shard_range
+    assert shard_range(64, 8, 4, 3) == (48, 64)
+    with pytest.raises(ValueError):
+        shard_range(64, 8, 3, 0)      # 64 tokens do not split over 3 ranks
+    with pytest.raises(ValueError):
+        shard_range(48, 16, 2, 0)     # 24 tokens per rank is not a whole number of 16-token groups
