@@ -467,6 +467,72 @@ def run_ours(args, w):
     return 0
 
 
+def run_sequence_sharded(args, w):
+    """--mode sequence: one sequence split across the ranks (whole groups per rank, the
+    shifted heads' G/2 halo exchanged between neighbours).  A step = RoPE-PI of the rank's
+    rows at their positions + sharded forward + sharded backward; the total work is fixed,
+    so "scaling" is "strong".  With one GPU the halo is the rank's own first rows, and the
+    number measures the cost of the local layout against the direct path."""
+    import torch
+    import torch.distributed as dist
+
+    import shifted_sparse_attention_s2attn_b200 as s2
+    from shifted_sparse_attention_s2attn_b200.sharded import shard_range, sharded_bwd, sharded_fwd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
+    t0, t1 = shard_range(w.N, w.G, world, rank)
+    host = {n: make_tensor(w, n)[:, t0:t1] for n in ("q", "k", "v", "dout")}
+    dv_ = {n: torch.from_numpy(np.ascontiguousarray(host[n]).view(np.int16)).view(torch.bfloat16).to(dev)
+           for n in host}
+    q, k = dv_["q"], dv_["k"]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        # in place every step, as in the replicas mode (the timing does not depend on the values)
+        s2.rope_pi_apply_offset(q, k, t0, w.pos_scale, w.base, stream)
+        o, lse = sharded_fwd(q, k, dv_["v"], w.G, w.shift_heads)
+        return sharded_bwd(q, k, dv_["v"], o, dv_["dout"], lse, w.G, w.shift_heads)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    s2.clear_device_error()
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    rc, detail = s2.get_device_error()
+    if rc != 0:
+        raise SystemExit(f"device error word set during the timed region: {detail:#x}")
+    ms_max = max_over_ranks(e0.elapsed_time(e1), dev)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    value = step_flops(w) * args.steps / (ms_max / 1e3) / 1e12   # the whole sequence's work, all ranks
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "mode": "sequence",
+            "config": dict(workload_config(w), parallelism=f"sequence x{world}",
+                           step="rope_pi_apply_offset + sharded fwd + sharded bwd (G/2 halo of the shifted heads)")}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -475,6 +541,9 @@ def main():
     ap.add_argument("--workload", default="llama2_7b_32k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "sequence"],
+                    help="replicas: every rank runs the whole workload (default); sequence: the "
+                         "workload's sequence is split across the ranks")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")
@@ -483,6 +552,8 @@ def main():
         raise SystemExit("the bench times the bf16 tensor-core path")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.mode == "sequence":
+        return run_sequence_sharded(args, w)
     return run_ours(args, w)
 
 
