@@ -130,3 +130,21 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(s2, "library_path", "/nonexistent/libs2attn.so")
     with pytest.raises(RuntimeError):
         s2.capi()
+
+
+def test_plain_c_caller(tmp_path, lib):
+    """The boundary is a C ABI: a C99 program built against include/s2attn.h and linked
+    with libs2attn.so runs its host-side checks (tests/c_abi/check_boundary.c)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    from shifted_sparse_attention_s2attn_b200 import library_path
+    libdir = os.path.dirname(library_path)
+    exe = tmp_path / "check_boundary"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi", "check_boundary.c"), "-o", str(exe), "-L", libdir,
+                    "-ls2attn", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
