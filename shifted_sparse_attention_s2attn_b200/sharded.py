@@ -16,14 +16,15 @@ Tokens belong to exactly one group per head, so results are moved, never summed.
 
 The exchanges are point-to-point sends and receives between ring neighbours through
 torch.distributed (NCCL over NVLink between GPUs; gloo on CPU).  A halo of G/2 rows is
-copied into this rank's memory before any kernel reads it.  The attention itself runs in
-`attn_fwd` / `attn_bwd`, by default this library's CUDA kernels; a caller can pass other
-callables with the same signatures (the CPU tests pass the oracle).
+copied into this rank's memory before any kernel reads it.  The steps are public:
+to_local (exchange and local layout), the kernels with shift_heads = 0, and to_owner
+(un-roll and return of the halo rows); sharded_fwd / sharded_bwd compose them with this
+library's CUDA kernels.
 """
 import torch
 import torch.distributed as dist
 
-__all__ = ["shard_range", "sharded_fwd", "sharded_bwd"]
+__all__ = ["shard_range", "to_local", "to_owner", "sharded_fwd", "sharded_bwd"]
 
 
 def shard_range(N, G, world, rank):
@@ -111,6 +112,37 @@ def _lse_from_local(lse_z, G, hs, group):
     return x
 
 
+def to_local(xs, G, shift_heads, group=None, lse=None):
+    """The local layout of this rank's inputs: the shifted heads of each [B, Np, H, D] tensor
+    in `xs` hold rows [G/2, Np) followed by the next rank's first G/2 rows, exchanged here;
+    the other heads are unchanged.  With `lse` ([B, H, Np]) its shifted heads are laid out
+    the same way.  Returns the list of local tensors (and the local lse when given)."""
+    B, Np, H, D = _check(xs[0], G, shift_heads)
+    hs, half = H - shift_heads, G // 2
+    if shift_heads == 0:
+        return (list(xs), lse) if lse is not None else list(xs)
+    sends = [x[:, :half, hs:] for x in xs] + ([lse[:, hs:, :half]] if lse is not None else [])
+    halos = _ring_shift(sends, -1, group)
+    zs = _to_local(xs, halos[: len(xs)], G, hs)
+    if lse is None:
+        return zs
+    return zs, _lse_to_local(lse, halos[len(xs)], G, hs)
+
+
+def to_owner(zs, G, shift_heads, group=None, lse=None):
+    """Undoes to_local for results computed on the local layout: each tensor's shifted heads
+    go back to this rank's rows, and the halo rows' results travel to the next rank, which
+    owns those tokens.  Returns the list of tensors (and the lse when given)."""
+    H = zs[0].shape[2]
+    hs = H - shift_heads
+    if shift_heads == 0:
+        return (list(zs), lse) if lse is not None else list(zs)
+    out = _from_local(list(zs), G, hs, group)
+    if lse is None:
+        return out
+    return out, _lse_from_local(lse, G, hs, group)
+
+
 def _cuda_fwd(q, k, v, G):
     from . import s2attn_fwd
     B, N, H, D = q.shape
@@ -129,32 +161,19 @@ def _cuda_bwd(q, k, v, o, dout, lse, G):
     return dq, dk, dv
 
 
-def sharded_fwd(q, k, v, G, shift_heads, group=None, attn_fwd=None):
-    """S^2-Attn forward on this rank's run of tokens ([B, Np, H, D] each).  Returns this
-    rank's o [B, Np, H, D] and lse [B, H, Np], equal to the rows [t0, t1) of the
-    unsharded call (shard_range gives t0, t1)."""
-    B, Np, H, D = _check(q, G, shift_heads)
-    attn_fwd = attn_fwd or _cuda_fwd
-    if shift_heads == 0:
-        return attn_fwd(q, k, v, G)
-    hs, half = H - shift_heads, G // 2
-    halos = _ring_shift([x[:, :half, hs:] for x in (q, k, v)], -1, group)
-    qz, kz, vz = _to_local((q, k, v), halos, G, hs)
-    oz, lse_z = attn_fwd(qz, kz, vz, G)
-    (o,) = _from_local([oz], G, hs, group)
-    return o, _lse_from_local(lse_z, G, hs, group)
+def sharded_fwd(q, k, v, G, shift_heads, group=None):
+    """S^2-Attn forward on this rank's run of tokens ([B, Np, H, D] bf16 CUDA tensors).
+    Returns this rank's o [B, Np, H, D] and lse [B, H, Np], equal to the rows [t0, t1) of
+    the unsharded call (shard_range gives t0, t1)."""
+    qz, kz, vz = to_local((q, k, v), G, shift_heads, group)
+    oz, lse_z = _cuda_fwd(qz, kz, vz, G)
+    (o,), lse = to_owner([oz], G, shift_heads, group, lse=lse_z)
+    return o, lse
 
 
-def sharded_bwd(q, k, v, o, dout, lse, G, shift_heads, group=None, attn_bwd=None):
+def sharded_bwd(q, k, v, o, dout, lse, G, shift_heads, group=None):
     """S^2-Attn backward on this rank's run of tokens: dq, dk, dv [B, Np, H, D], equal to
     the rows [t0, t1) of the unsharded backward."""
-    B, Np, H, D = _check(q, G, shift_heads)
-    attn_bwd = attn_bwd or _cuda_bwd
-    if shift_heads == 0:
-        return attn_bwd(q, k, v, o, dout, lse, G)
-    hs, half = H - shift_heads, G // 2
-    halos = _ring_shift([x[:, :half, hs:] for x in (q, k, v, o, dout)] + [lse[:, hs:, :half]], -1, group)
-    qz, kz, vz, oz, dz = _to_local((q, k, v, o, dout), halos[:5], G, hs)
-    lse_z = _lse_to_local(lse, halos[5], G, hs)
-    dqz, dkz, dvz = attn_bwd(qz, kz, vz, oz, dz, lse_z, G)
-    return tuple(_from_local([dqz, dkz, dvz], G, hs, group))
+    (qz, kz, vz, oz, dz), lse_z = to_local((q, k, v, o, dout), G, shift_heads, group, lse=lse)
+    dqz, dkz, dvz = _cuda_bwd(qz, kz, vz, oz, dz, lse_z, G)
+    return tuple(to_owner([dqz, dkz, dvz], G, shift_heads, group))

@@ -1,7 +1,9 @@
-"""Sequence-sharded S^2-Attn on CPU: gloo ranks exchange the G/2 halos of the shifted heads,
-run the per-rank attention (here the fp64 oracle, with shift_heads = 0 on the local
-layout), and the rows they return, put side by side, must equal the oracle on the whole
-sequence with the shift -- forward (o, lse) and backward (dq, dk, dv)."""
+"""Sequence-sharded S^2-Attn on CPU: gloo ranks exchange the G/2 halos of the shifted heads
+(to_local), the test runs the fp64 oracle with shift_heads = 0 on each rank's local layout,
+and the results go back to their owners (to_owner); the rows, put side by side, must equal
+the oracle on the whole sequence with the shift -- forward (o, lse) and backward (dq, dk,
+dv).  The library's sharded_fwd / sharded_bwd compose the same steps with the CUDA kernels
+(tests/test_gpu_sharded.py)."""
 import os
 import socket
 
@@ -26,29 +28,22 @@ def _inputs():
     return [rng.standard_normal((B, N, H, D)) for _ in range(4)]
 
 
-def _oracle_fwd(q, k, v, G):
-    import oracle
-    o, lse = oracle.s2attn_fwd(q.numpy(), k.numpy(), v.numpy(), G, 0)
-    return torch.from_numpy(o), torch.from_numpy(lse)
-
-
-def _oracle_bwd(q, k, v, o, dout, lse, G):
-    import oracle
-    # the o and lse handed over must be those of the local layout (they travel through the halo exchange)
-    o_ref, lse_ref = oracle.s2attn_fwd(q.numpy(), k.numpy(), v.numpy(), G, 0)
-    assert np.abs(o.numpy() - o_ref).max() < 1e-12 and np.abs(lse.numpy() - lse_ref).max() < 1e-12
-    dq, dk, dv = oracle.s2attn_bwd(q.numpy(), k.numpy(), v.numpy(), dout.numpy(), G, 0)
-    return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv)
-
-
 def _run_rank(rank, world):
     import sys
     sys.path.insert(0, ROOT)
-    from shifted_sparse_attention_s2attn_b200.sharded import shard_range, sharded_bwd, sharded_fwd
+    import oracle
+    from shifted_sparse_attention_s2attn_b200.sharded import shard_range, to_local, to_owner
     t0, t1 = shard_range(N, G, world, rank)
     q, k, v, do = (torch.from_numpy(x[:, t0:t1].copy()) for x in _inputs())
-    o, lse = sharded_fwd(q, k, v, G, SH, attn_fwd=_oracle_fwd)
-    dq, dk, dv = sharded_bwd(q, k, v, o, do, lse, G, SH, attn_bwd=_oracle_bwd)
+    # forward: local layout, oracle with shift 0, results back to their owners
+    qz, kz, vz = to_local((q, k, v), G, SH)
+    oz, lse_z = (torch.from_numpy(a) for a in oracle.s2attn_fwd(qz.numpy(), kz.numpy(), vz.numpy(), G, 0))
+    (o,), lse = to_owner([oz], G, SH, lse=lse_z)
+    # backward: o and lse travel through the exchange too; they must come back as the local layout's
+    (qz2, kz2, vz2, oz2, dz), lse_z2 = to_local((q, k, v, o, do), G, SH, lse=lse)
+    assert torch.equal(oz2, oz) and torch.equal(lse_z2, lse_z)
+    grads = oracle.s2attn_bwd(qz2.numpy(), kz2.numpy(), vz2.numpy(), dz.numpy(), G, 0)
+    dq, dk, dv = to_owner([torch.from_numpy(a) for a in grads], G, SH)
     return [x.numpy() for x in (o, lse, dq, dk, dv)]
 
 
