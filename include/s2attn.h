@@ -191,7 +191,10 @@ int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* 
 /*
  * Reads the current device's error word: S2ATTN_OK if no kernel has failed since
  * the last clear, else S2ATTN_ERR_DEVICE_TIMEOUT with *detail (if non-NULL) set to
- * (kernel << 8) | site (kernel 1 = forward, 2 = backward, 4 = decoding step).  Synchronize the streams
+ * (kernel << 8) | site (kernel 1 = forward, 2 = backward, 4 = decoding step).  In the
+ * bounds-checked build (libs2attn_debug.so, compiled with S2ATTN_DEBUG) a site with bit
+ * 0x80 set is a global store or reduction whose computed index fell outside its tensor;
+ * the access was skipped.  Synchronize the streams
  * that ran library kernels first.
  */
 int s2attn_get_device_error(int* detail);

@@ -17,7 +17,8 @@ __all__ = [
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_HERE, "libs2attn.so")
+# S2ATTN_LIBRARY selects another build of the library, e.g. libs2attn_debug.so (bounds-checked)
+library_path = os.environ.get("S2ATTN_LIBRARY") or os.path.join(_HERE, "libs2attn.so")
 
 STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "workspace", -4: "CUDA error",
           -5: "device timeout"}

@@ -312,4 +312,24 @@ __device__ __forceinline__ void report_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// ---- debug builds (-DS2ATTN_DEBUG): bounds checks of computed global addresses ----
+// The stand-in for a memory checker: every global store or reduction whose index is
+// computed (from tiles, groups, the roll, splits) is checked against its tensor's extent.
+#ifdef S2ATTN_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+constexpr int kDebugSite = 0x80;
+
+// True when elements [first, first + count) lie inside [0, limit).  Otherwise, in debug
+// builds, records (code | kDebugSite) in the error word and returns false so that the
+// caller skips the access.  Release builds compile the check away.
+__device__ __forceinline__ bool in_bounds(size_t first, size_t count, size_t limit, int* err, int code) {
+  if (!kDebugChecks) return true;
+  if (first + count <= limit) return true;
+  report_error(err, code | kDebugSite);
+  return false;
+}
+
 }  // namespace s2

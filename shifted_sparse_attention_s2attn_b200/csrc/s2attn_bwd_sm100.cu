@@ -99,8 +99,9 @@ __device__ __forceinline__ void issue_kq(uint32_t d, uint32_t sa, uint32_t sb, u
   }
 }
 
-// Stores one 128-column fp32 accumulator row (TMEM) as bf16, times `mul`, to global memory.
-__device__ __forceinline__ void store_row_bf16(uint32_t taddr, __nv_bfloat16* dst_row, float mul) {
+// Stores one 128-column fp32 accumulator row (TMEM) as bf16, times `mul`, to global memory
+// (the TMEM loads are warp-collective and always run; `store` gates the global writes).
+__device__ __forceinline__ void store_row_bf16(uint32_t taddr, __nv_bfloat16* dst_row, float mul, bool store) {
 #pragma unroll
   for (int c = 0; c < HD; c += 32) {
     uint32_t r[32], pk[16];
@@ -109,8 +110,10 @@ __device__ __forceinline__ void store_row_bf16(uint32_t taddr, __nv_bfloat16* ds
     for (int e = 0; e < 16; ++e)
       pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
     uint4* dst = reinterpret_cast<uint4*>(dst_row + c);
+    if (store) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+    }
   }
 }
 
@@ -489,10 +492,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const int tok = token_of(kt * BK) + kr;
+      const size_t row_first = ((size_t)(b * p.N + tok) * p.H + h) * HD;
+      const bool row_ok = in_bounds(row_first, HD, (size_t)p.B * p.N * p.H * HD, p.err, (K_BWD << 8) | SITE_PDS);
       if (hf == 0)
-        store_row_bf16(lane_addr + TM_DK, p.dk + ((size_t)(b * p.N + tok) * p.H + h) * HD, p.scale);
+        store_row_bf16(lane_addr + TM_DK, p.dk + row_first, p.scale, row_ok);
       else
-        store_row_bf16(lane_addr + TM_DV, p.dv + ((size_t)(b * p.N + tok) * p.H + h) * HD, 1.0f);
+        store_row_bf16(lane_addr + TM_DV, p.dv + row_first, 1.0f, row_ok);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dkv_empty);
@@ -520,6 +525,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // query q of this tile -> dq_acc[b, tok0 + q, h, d]; a warp covers 32 consecutive d (128 B)
         float* dst = p.dq_acc + ((size_t)(b * p.N + token_of((kt + s) * BQ)) * p.H + h) * HD + d;
         const size_t row_stride = (size_t)p.H * HD;
+#ifdef S2ATTN_DEBUG
+        // the 128 queries of the tile: dst + q * row_stride for q < 128 (the release build keeps
+        // this path free of the check: the drain's registers are at their limit)
+        const bool dq_ok = in_bounds((size_t)(dst - p.dq_acc), (BQ - 1) * row_stride + 1,
+                                     (size_t)p.B * p.N * p.H * HD, p.err, (K_BWD << 8) | SITE_DQ);
+#else
+        constexpr bool dq_ok = true;
+#endif
         uint32_t r0[64], r1[64];
         tmem_ld_x64(lane_addr + TM_DP, r0);
         tmem_ld_x64(lane_addr + TM_DP + 64, r1);
@@ -528,15 +541,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(dq_free);
         // one running address (consecutive queries are row_stride floats apart)
+        if (dq_ok) {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          red_add_f32(dst, __uint_as_float(r0[e]));
-          dst += row_stride;
-        }
+          for (int e = 0; e < 64; ++e) {
+            red_add_f32(dst, __uint_as_float(r0[e]));
+            dst += row_stride;
+          }
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          red_add_f32(dst, __uint_as_float(r1[e]));
-          dst += row_stride;
+          for (int e = 0; e < 64; ++e) {
+            red_add_f32(dst, __uint_as_float(r1[e]));
+            dst += row_stride;
+          }
         }
       }
     }

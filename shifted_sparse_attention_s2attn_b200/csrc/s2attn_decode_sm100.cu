@@ -309,8 +309,10 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 2)
         o += wgt * wo[(w * MT + m) * HD + d];
       }
     }
-    p.part_o[(part * p.M + m) * HD + d] = o;
-    if (d == 0) {
+    const size_t n_parts = (size_t)p.B * p.H * p.S * p.M;
+    if (in_bounds((part * p.M + m) * HD + d, 1, n_parts * HD, p.err, (K_DEC << 8) | SITE_CONSUME))
+      p.part_o[(part * p.M + m) * HD + d] = o;
+    if (d == 0 && in_bounds((part * p.M + m) * 2, 2, n_parts * 2, p.err, (K_DEC << 8) | SITE_CONSUME)) {
       p.part_ml[(part * p.M + m) * 2] = mx;
       p.part_ml[(part * p.M + m) * 2 + 1] = l;
     }
@@ -672,11 +674,14 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       // partial of this split: unnormalised O row, running max (log2 domain) and sum
       tc_fence_after();
       const size_t part = (size_t)bh * p.S + split;
+      const size_t n_parts = (size_t)p.B * p.H * p.S * p.M;
+      const bool row_ok = r < p.M && in_bounds((part * p.M + r) * HD, HD, n_parts * HD, p.err,
+                                                 (K_DEC << 8) | SITE_SOFTMAX);
 #pragma unroll
       for (int c = 0; c < HD; c += 32) {
         uint32_t rr[32];
         tmem_ld_x32(lane_addr + TM_O + c, rr);
-        if (r < p.M) {
+        if (row_ok) {
           float4* dst = reinterpret_cast<float4*>(p.part_o + (part * p.M + r) * HD + c);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
@@ -684,7 +689,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
                                  __uint_as_float(rr[4 * e + 2]), __uint_as_float(rr[4 * e + 3]));
         }
       }
-      if (r < p.M) {
+      if (row_ok) {
         p.part_ml[(part * p.M + r) * 2] = m_run;
         p.part_ml[(part * p.M + r) * 2 + 1] = l_run;
       }

@@ -387,7 +387,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       const int tok = tile_token0(qt) + row;
       const float inv_l = 1.0f / l_run;
-      __nv_bfloat16* orow = p.o + ((size_t)(b * p.N + tok) * p.H + h) * HD;
+      const size_t o_first = ((size_t)(b * p.N + tok) * p.H + h) * HD;
+      const size_t lse_idx = ((size_t)b * p.H + h) * p.N + tok;
+      const bool o_ok = in_bounds(o_first, HD, (size_t)p.B * p.N * p.H * HD, p.err, (K_FWD << 8) | SITE_EPILOGUE);
+      const bool lse_ok = in_bounds(lse_idx, 1, (size_t)p.B * p.H * p.N, p.err, (K_FWD << 8) | SITE_EPILOGUE);
+      __nv_bfloat16* orow = p.o + o_first;
 #pragma unroll
       for (int c = 0; c < HD; c += 32) {
         uint32_t r[32];
@@ -397,10 +401,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
         uint4* dst = reinterpret_cast<uint4*>(orow + c);
+        if (o_ok) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
       }
-      p.lse[((size_t)b * p.H + h) * p.N + tok] = (m_run + log2f(l_run)) * LN2;
+      if (lse_ok) p.lse[lse_idx] = (m_run + log2f(l_run)) * LN2;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_empty[i]);

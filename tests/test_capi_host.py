@@ -148,3 +148,12 @@ def test_plain_c_caller(tmp_path, lib):
                     "-ls2attn", f"-Wl,-rpath,{libdir}"], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
+
+
+def test_debug_build_exports_the_same_boundary(lib):
+    """The bounds-checked build (libs2attn_debug.so, -DS2ATTN_DEBUG) is the same C ABI."""
+    from shifted_sparse_attention_s2attn_b200 import _build
+    debug = ctypes.CDLL(_build.build(debug=True))
+    for name in _declared_functions():
+        assert hasattr(debug, name), name
+    assert debug.s2attn_version() == 100
