@@ -426,17 +426,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_ld_x64(lane_addr + TM_S + 64 * hf, sr);
           // on the diagonal tile (s == 0) query column c of the tile is visible iff c >= key row
           const int lim = (s == 0) ? kr - 64 * hf : -1;
+          const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
           for (int c4 = 0; c4 < 16; ++c4) {
             const float4 l4 = reinterpret_cast<const float4*>(lse_s)[c4];  // -lse * log2(e)
-            const float nl[4] = {l4.x, l4.y, l4.z, l4.w};
-            float pv[4];
+            // s * scale * log2(e) - lse * log2(e), two elements per packed fp32x2 FMA
+            const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1])),
+                                          sl2x2, make_float2(l4.x, l4.y));
+            const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
+                                          sl2x2, make_float2(l4.z, l4.w));
+            float pv[4] = {ex2_approx(x01.x), ex2_approx(x01.y), ex2_approx(x23.x), ex2_approx(x23.y)};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 4 * c4 + e;
-              pv[e] = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, nl[e]));
-              if (c < lim) pv[e] = 0.0f;
-            }
+            for (int e = 0; e < 4; ++e)
+              if (4 * c4 + e < lim) pv[e] = 0.0f;
             pp[2 * c4] = pack_bf16x2(pv[0], pv[1]);
             pp[2 * c4 + 1] = pack_bf16x2(pv[2], pv[3]);
           }
@@ -472,11 +474,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int c4 = 0; c4 < 8; ++c4) {
             const float4 d4 = reinterpret_cast<const float4*>(delta_s)[8 * half + c4];
-            pk[2 * c4] = mul_bf16x2(pp[16 * half + 2 * c4], pack_bf16x2(__uint_as_float(dr[4 * c4]) - d4.x,
-                                                                      __uint_as_float(dr[4 * c4 + 1]) - d4.y));
-            pk[2 * c4 + 1] = mul_bf16x2(pp[16 * half + 2 * c4 + 1],
-                                        pack_bf16x2(__uint_as_float(dr[4 * c4 + 2]) - d4.z,
-                                                    __uint_as_float(dr[4 * c4 + 3]) - d4.w));
+            // dP - delta, two elements per packed fp32x2 add
+            const float2 g01 = __fadd2_rn(make_float2(__uint_as_float(dr[4 * c4]), __uint_as_float(dr[4 * c4 + 1])),
+                                          make_float2(-d4.x, -d4.y));
+            const float2 g23 = __fadd2_rn(make_float2(__uint_as_float(dr[4 * c4 + 2]), __uint_as_float(dr[4 * c4 + 3])),
+                                          make_float2(-d4.z, -d4.w));
+            pk[2 * c4] = mul_bf16x2(pp[16 * half + 2 * c4], pack_bf16x2(g01.x, g01.y));
+            pk[2 * c4 + 1] = mul_bf16x2(pp[16 * half + 2 * c4 + 1], pack_bf16x2(g23.x, g23.y));
           }
 #pragma unroll
           for (int c = 0; c < 4; ++c)
