@@ -10,7 +10,8 @@ SDPA in fp64) for G=N without shift; brute force with an explicit N x N mask for
 grouped and shifted heads; the shift example of the "LongLoRA paper notes" page
 (section 3.3); central finite differences for the gradients; RoPE invariants; for the
 decoding step, torch SDPA with an explicit mask, the last rows of full causal
-attention, and closed forms.
+attention, and closed forms.  The LoRA-adapted projection (lora.py, numpy fp64) is pinned
+by tests/test_oracle_lora_pins.py.
 """
 import ctypes
 import numpy as np
@@ -167,3 +168,5 @@ def rope_pi_bf16_at(x_bits, pos0, pos_scale, base=10000.0):
     _load().oracle_rope_pi_f32_bf16_at(_ptr(x), _ptr(y), B, N, H, D, int(pos0), float(pos_scale), float(base))
     return y
 
+
+from .lora import lora_proj  # noqa: E402  (numpy fp64; see lora.py)

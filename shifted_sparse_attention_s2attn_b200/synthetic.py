@@ -108,3 +108,34 @@ def scaled(w: Workload, **changes) -> Workload:
     d = dict(w.__dict__)
     d.update(changes)
     return Workload(**d)
+
+
+# ---- LoRA-adapted projections ------------------------------------------------------
+# The LLaMA2-7B layer: hidden size 4096 = H*D (32 heads of 128); q, k, v stacked (parts 3)
+# and o (parts 1); LoRA rank 8 with alpha 16 (scaling 2), LongLoRA's adapter setting.
+LORA_LLAMA2_7B = dict(K=4096, n_out=4096, r=8, scaling=2.0)
+LORA_IDS = {"x": 10, "w": 11, "a": 12, "b": 13}
+
+
+def make_lora_inputs(T, K, n_out, parts, r, seed=0, b_std=0.05):
+    """Seeded inputs of a LoRA-adapted projection, as bf16 bit patterns (uint16).
+
+    numpy.random.default_rng(1000*seed + id) draws standard normals in fp32 (ids: x 10,
+    W 11, A 12, B 13), scaled and rounded to bf16 (nearest even):
+      x [T, K]             ~ N(0, 1)          (a layer's normalised hidden states)
+      W [parts*n_out, K]   ~ N(0, 1/K)        (so every output is ~ N(0, 1))
+      A [parts*r, K]       ~ N(0, 1/K)
+      B [parts*n_out, r]   ~ N(0, b_std^2)    (nonzero, as after some training; LoRA
+                                               starts B at zero, which would hide the term)
+    Returns (x, W, A, B); A and B are None when r == 0."""
+    def draw(name, shape, std):
+        rng = np.random.default_rng(1000 * seed + LORA_IDS[name])
+        x = rng.standard_normal(shape, dtype=np.float32)
+        if std != 1.0:
+            x *= np.float32(std)
+        return f32_to_bf16_bits(x)
+    x = draw("x", (T, K), 1.0)
+    w = draw("w", (parts * n_out, K), 1.0 / np.sqrt(K))
+    if r == 0:
+        return x, w, None, None
+    return x, w, draw("a", (parts * r, K), 1.0 / np.sqrt(K)), draw("b", (parts * n_out, r), b_std)
