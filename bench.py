@@ -359,6 +359,43 @@ def run_ours(args, w):
                            "tokens_per_s": B * M / (d_ms / 1e3)}
         del dq_, d_o, d_lse, d_ws
 
+    # ---- LoRA-adapted projections on either side of the attention (LLaMA2-7B layer) ----
+    # q, k, v stacked (3 x 4096 outputs, rank 8, scaling 2, RoPE-PI fused on q and k) and o
+    # (4096 outputs, rank 8) over the B*N tokens; the plain q, k, v projection (no adapter,
+    # no RoPE) is timed too, to show what the adapter and the rotation add.
+    lora = {}
+    T_l, K_l, n_l, r_l = B * N, H * D, H * D, 8
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20)
+    lx = torch.randn((T_l, K_l), generator=gen, device=dev).to(torch.bfloat16)
+    for name, parts, r_, rope_parts in (("qkv_lora_rope", 3, r_l, 2), ("qkv_plain", 3, 0, 0), ("o_lora", 1, r_l, 0)):
+        lw = (torch.randn((parts * n_l, K_l), generator=gen, device=dev) / K_l ** 0.5).to(torch.bfloat16)
+        la = (torch.randn((parts * r_, K_l), generator=gen, device=dev) / K_l ** 0.5).to(torch.bfloat16) if r_ else None
+        lb = (0.05 * torch.randn((parts * n_l, r_), generator=gen, device=dev)).to(torch.bfloat16) if r_ else None
+        ly = torch.empty((parts, T_l, n_l), dtype=torch.bfloat16, device=dev)
+        lws = torch.empty(max(256, s2.lora_proj_workspace_bytes(T_l, K_l, n_l, parts, r_)), dtype=torch.uint8,
+                          device=dev)
+        call = lambda: s2.lora_proj_fwd(lx, lw, la, lb, ly, parts, 2.0, rope_parts=rope_parts, head_dim=D,  # noqa: E731
+                                        seq_len=N, pos_scale=w.pos_scale, workspace=lws, stream=stream)
+        for _ in range(3):
+            call()
+        l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        l_reps = 10
+        l0.record(stream)
+        for _ in range(l_reps):
+            call()
+        l1.record(stream)
+        torch.cuda.synchronize(dev)
+        l_ms = l0.elapsed_time(l1) / l_reps
+        flops = 2 * T_l * K_l * parts * n_l + 2 * T_l * K_l * parts * r_ + 2 * T_l * r_ * parts * n_l
+        lora[name] = {"ms": l_ms, "parts": parts, "r": r_, "rope_parts": rope_parts, "flops": flops,
+                      "tflops": flops / (l_ms / 1e3) / 1e12}
+        del lw, la, lb, ly, lws
+    del lx
+    rc, detail = s2.get_device_error()
+    if rc != 0:
+        raise SystemExit(f"device error word set during the projection runs: {detail:#x}")
+
     # ---- end to end: host buffers in, results out, through the same public calls ----
     # Each step copies its inputs from pinned host memory and its results back.  Steps are
     # pipelined over three streams with two device buffer sets: the host->device copy of
@@ -458,6 +495,13 @@ def run_ours(args, w):
                    "bound": "hbm", "peak_gbs": peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]),
                    **{k_: dict(v_, frac=v_["gbs"] / peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
                       for k_, v_ in decode.items()}},
+        "lora_proj": {"workload": f"LLaMA2-7B layer projections over T=B*N={B * N} tokens, K={H * D}: q,k,v "
+                                  f"stacked (3x{H * D} outputs) and o ({H * D}); LoRA rank 8, scaling 2; RoPE-PI "
+                                  f"(pos_scale {w.pos_scale}) fused on q and k; flops = 2*T*K*outputs + adapter",
+                      "bound": "tensor", "peak": peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
+                      "peak_source": f"{peak_src} bf16_tflops (burst: each call timed alone, 10 calls)",
+                      **{k_: dict(v_, frac=v_["tflops"] / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+                         for k_, v_ in lora.items()}},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks,
     }

@@ -164,6 +164,40 @@ int rope_pi_apply_offset(void* q, void* k, int B, int N, int H, int D, int pos0,
                          void* stream);
 
 /*
+ * LoRA-adapted linear projections, the steps on either side of S^2-Attn in a LongLoRA
+ * layer ("LongLoRA paper notes", section 3.2: low-rank adapters on the Q, K, V and O
+ * projections; nearauto.com article, "long-context LoRA improvement").  For `parts`
+ * projections stacked along the output (3 for q, k, v; 1 for o), part p computes
+ *   y[p] = x W_p^T + scaling * (x A_p^T) B_p^T
+ * and the first `rope_parts` parts are then rotated by RoPE-PI, so q and k come out ready
+ * for s2attn_fwd.  All bf16, accumulated in fp32 on the tensor cores:
+ *   x      : [T, K], T = B*seq_len tokens (row t is position t mod seq_len)
+ *   w      : [parts*n_out, K], the frozen weights (the layout of a linear layer's weight)
+ *   lora_a : [parts*r, K], the adapters' down projections (NULL when r == 0)
+ *   lora_b : [parts*n_out, r], the adapters' up projections (NULL when r == 0)
+ *   y      : [parts, T, n_out] output; y[p] is a contiguous [B, seq_len, H, D] tensor when
+ *            n_out = H*D, so q, k and v need no copy before attention
+ * Rounding: the rank-r intermediate is held in bf16 after scaling, bf16(scaling * x A_p^T),
+ * and y is rounded once (nearest even) from the fp32 accumulator.  With rope_parts > 0,
+ * the rotated parts are bit-identical to this call with rope_parts = 0 followed by
+ * rope_pi_apply(y[p], ..., B, seq_len, n_out/head_dim, head_dim, pos_scale, base) on
+ * each: the same table (cached per device, seq_len, head_dim, pos_scale, base) and the
+ * same fp32 operation order, applied to the bf16-rounded projection.
+ * Requirements: K >= 8 and K % 8 == 0; 0 <= r <= 64; 0 <= rope_parts <= parts;
+ * n_out % 256 == 0 (else S2ATTN_ERR_UNSUPPORTED); x, w, y, lora_a 16-byte aligned; with
+ * rope_parts > 0: head_dim in {32, 64, 128, 256}, T % seq_len == 0, base > 0.
+ * `workspace` (device, caller-owned, 256-byte aligned, at least
+ * lora_proj_workspace_bytes(T, K, n_out, parts, r) bytes; may be NULL when r == 0) holds the
+ * zero-padded adapters and the intermediate and is overwritten.  Runs up to three kernels
+ * on `stream` (adapter padding, the rank-r down projection, the projection); invalid
+ * arguments return before any launch.
+ */
+size_t lora_proj_workspace_bytes(int T, int K, int n_out, int parts, int r);
+int lora_proj_fwd(const void* x, const void* w, const void* lora_a, const void* lora_b, void* y, int T, int K,
+                  int n_out, int parts, int r, float scaling, int rope_parts, int head_dim, int seq_len,
+                  float pos_scale, float base, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Backward pass that allocates nothing.  The LongLoRA pages have no counterpart of
  * this entry point; it exists for callers that cannot allocate device memory on
  * the call path (a runtime whose allocator already holds the device's memory, a
@@ -191,7 +225,8 @@ int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* 
 /*
  * Reads the current device's error word: S2ATTN_OK if no kernel has failed since
  * the last clear, else S2ATTN_ERR_DEVICE_TIMEOUT with *detail (if non-NULL) set to
- * (kernel << 8) | site (kernel 1 = forward, 2 = backward, 4 = decoding step).  In the
+ * (kernel << 8) | site (kernel 1 = forward, 2 = backward, 4 = decoding step,
+ * 5 = LoRA projection).  In the
  * bounds-checked build (libs2attn_debug.so, compiled with S2ATTN_DEBUG) a site with bit
  * 0x80 set is a global store or reduction whose computed index fell outside its tensor;
  * the access was skipped.  Synchronize the streams

@@ -13,6 +13,7 @@ __all__ = [
     "S2AttnError", "capi", "library_path",
     "s2attn_fwd", "s2attn_bwd", "s2attn_bwd_workspace_bytes", "s2attn_bwd_preprocess", "s2attn_bwd_main",
     "s2attn_bwd_dq_convert", "s2attn_bwd_noalloc", "s2attn_decode", "s2attn_decode_workspace_bytes", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply", "rope_pi_apply_offset",
+    "lora_proj_fwd", "lora_proj_workspace_bytes",
     "get_device_error", "clear_device_error", "s2attn_selftest_bounded_wait",
 ]
 
@@ -59,6 +60,8 @@ def capi():
         "s2attn_bwd_f32": ([P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, P, Z, P], I),
         "rope_pi_apply": ([P, P, I, I, I, I, F, F, P], I),
         "rope_pi_apply_offset": ([P, P, I, I, I, I, I, F, F, P], I),
+        "lora_proj_workspace_bytes": ([I, I, I, I, I], Z),
+        "lora_proj_fwd": ([P, P, P, P, P, I, I, I, I, I, F, I, I, I, F, F, P, Z, P], I),
         "s2attn_get_device_error": ([ctypes.POINTER(I)], I),
         "s2attn_clear_device_error": ([], I),
         "s2attn_selftest_bounded_wait": ([ctypes.c_uint, P], I),
@@ -187,6 +190,33 @@ def rope_pi_apply_offset(q, k, pos0, pos_scale, base=10000.0, stream=None):
     B, N, H, D = _bnhd(ref, "q/k")
     _check("rope_pi_apply_offset", capi().rope_pi_apply_offset(_ptr(q), _ptr(k), B, N, H, D, int(pos0),
                                                                float(pos_scale), float(base), _stream(stream)))
+
+
+def lora_proj_workspace_bytes(T, K, n_out, parts, r):
+    return int(capi().lora_proj_workspace_bytes(T, K, n_out, parts, r))
+
+
+def lora_proj_fwd(x, w, lora_a, lora_b, y, parts, scaling, rope_parts=0, head_dim=128, seq_len=None,
+                  pos_scale=1.0, base=10000.0, workspace=None, stream=None):
+    """LoRA-adapted projections: y[p] = x W_p^T + scaling (x A_p^T) B_p^T for p < parts, RoPE-PI
+    on the first rope_parts parts.  x: [..., K] (T rows), w: [parts*n_out, K], lora_a:
+    [parts*r, K] and lora_b: [parts*n_out, r] (both None for r = 0), y: [parts, T, n_out]
+    (or any contiguous tensor of that many elements); all bf16 on the device.  workspace:
+    uint8 device tensor of lora_proj_workspace_bytes(T, K, n_out, parts, r) bytes (r > 0)."""
+    for t, name in ((x, "x"), (w, "w"), (y, "y"), (lora_a, "lora_a"), (lora_b, "lora_b")):
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    K = x.shape[-1]
+    T = x.numel() // K
+    n_out = w.shape[0] // parts
+    r = 0 if lora_a is None else lora_a.shape[0] // parts
+    if y.numel() != parts * T * n_out:
+        raise ValueError("y must hold parts * T * n_out elements")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("lora_proj_fwd", capi().lora_proj_fwd(
+        _ptr(x), _ptr(w), _ptr(lora_a), _ptr(lora_b), _ptr(y), T, K, n_out, parts, r, float(scaling),
+        int(rope_parts), int(head_dim), int(seq_len if seq_len is not None else T), float(pos_scale), float(base),
+        _ptr(workspace), ws_bytes, _stream(stream)))
 
 
 def get_device_error():

@@ -10,7 +10,7 @@ namespace s2 {
 
 // Device error codes (first failure wins; read with s2attn_get_device_error).
 // code = (kernel << 8) | site
-enum Kernel : int { K_FWD = 1, K_BWD = 2, K_SELFTEST = 3, K_DEC = 4 };
+enum Kernel : int { K_FWD = 1, K_BWD = 2, K_SELFTEST = 3, K_DEC = 4, K_LORA = 5 };
 
 // Problem description after validation.  Rows of a [B,N,H,D] tensor for head h
 // are addressed through 3-D tensor maps with dims {D, H, B*N}.
@@ -64,6 +64,27 @@ int decode_splits(int B, int N, int H, int n_sm, int* tiles_per_split);
 cudaError_t launch_decode_sm100(const CUtensorMap& tk, const CUtensorMap& tv, const void* q, void* o, float* lse,
                                 float* part_o, float* part_ml, int B, int M, int N, int H, int S,
                                 int tiles_per_split, int* err, cudaStream_t st);
+
+// LoRA-adapted projections y = x W^T + s (x A^T) B^T (lora_proj_sm100.cu).  The rank
+// dimension is zero-padded to kLoraRankPad (one 64-wide K block); the projection's output
+// tile is kLoraProjTileN columns, so n_out must be a multiple of it.
+constexpr int kLoraRankPad = 64;
+constexpr int kLoraMaxRank = kLoraRankPad;
+constexpr int kLoraProjTileN = 256;
+// a [parts*r, K], b [parts*n_out, r] -> a_pad [parts*64, K], b_pad [parts*n_out, 64] (zeros beyond r).
+cudaError_t launch_lora_pad(const void* a, const void* b, void* a_pad, void* b_pad, int parts, int r, int K,
+                            int n_out, cudaStream_t st);
+// u [parts, T, 64] = bf16(scaling * x a_pad^T).  Tensor maps (128-byte swizzle, 64-column
+// boxes): tx over x [T, K] with 128-row boxes, ta_pad over a_pad with 64-row boxes.
+cudaError_t launch_lora_down(const CUtensorMap& tx, const CUtensorMap& ta_pad, void* u, int T, int K, int parts,
+                             float scaling, int n_sm, int* err, cudaStream_t st);
+// y [parts, T, n_out] = bf16(x W^T + u_part b_pad^T), RoPE-PI on parts [0, rope_parts).
+// Tensor maps: tx as above; tw over W [parts*n_out, K] with 256-row boxes; tu over u as
+// {64, T, parts} with {64, 128, 1} boxes; tb over b_pad with 256-row boxes (r == 0: tu, tb unused).
+cudaError_t launch_lora_proj(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& tu,
+                             const CUtensorMap& tb, void* y, int T, int K, int n_out, int parts, int r,
+                             int rope_parts, int head_dim, int seq_len, const float* cos_tab, const float* sin_tab,
+                             int n_sm, int* err, cudaStream_t st);
 
 // RoPE-PI in place on bf16 q and k, with a cos/sin table [N, D/2] (fp32 each).
 cudaError_t launch_rope_pi(void* q, void* k, const float* cos_tab, const float* sin_tab, int B, int N, int H,

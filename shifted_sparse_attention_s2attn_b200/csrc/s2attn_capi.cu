@@ -70,6 +70,24 @@ bool map_bf16_sw128(CUtensorMap* m, const void* base, const s2::Shape& s, uint32
                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// A row-major bf16 matrix [outer, inner] (rank 2), or a stack [d2, outer, inner] (rank 3,
+// boxes one matrix deep), with 128-byte swizzled boxes of box_inner x box_outer elements;
+// out-of-range elements read as zero.  The rank must match the kernel's load instruction.
+bool map_rows_bf16(CUtensorMap* m, const void* base, int rank, uint64_t inner, uint64_t outer, uint64_t d2,
+                   uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, outer, d2};
+  cuuint64_t strides[2] = {inner * 2, inner * outer * 2};
+  cuuint32_t box[3] = {box_inner, box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (rank != 2 && rank != 3) return false;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---- validation -----------------------------------------------------------------
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -202,6 +220,9 @@ int decode_max_splits(int N) {
   const int tiles = (N + s2::kDecodeTileKeys - 1) / s2::kDecodeTileKeys;
   return tiles < s2::kDecodeMaxSplits ? tiles : s2::kDecodeMaxSplits;
 }
+
+// LoRA workspace: u [parts, T, 64] bf16, then a_pad, then b_pad (each 256-byte aligned).
+size_t lora_u_bytes(int T, int parts) { return align256((size_t)parts * T * s2::kLoraRankPad * 2); }
 
 size_t decode_part_o_bytes(int B, int M, int N, int H, int D) {
   return align256((size_t)B * H * decode_max_splits(N) * M * D * sizeof(float));
@@ -401,6 +422,67 @@ int rope_pi_apply_offset(void* q, void* k, int B, int N, int H, int D, int pos0,
   const size_t off = (size_t)pos0 * (D / 2);
   return cuda_status(s2::launch_rope_pi(q, k, tab.cos_d + off, tab.sin_d + off, B, N, H, D,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+size_t lora_proj_workspace_bytes(int T, int K, int n_out, int parts, int r) {
+  if (T < 1 || K < 1 || n_out < 1 || parts < 1 || r < 0 || r > s2::kLoraMaxRank) return 0;
+  if (r == 0) return 0;
+  return lora_u_bytes(T, parts) + align256((size_t)parts * s2::kLoraRankPad * K * 2) +
+         align256((size_t)parts * n_out * s2::kLoraRankPad * 2);
+}
+
+int lora_proj_fwd(const void* x, const void* w, const void* lora_a, const void* lora_b, void* y, int T, int K,
+                  int n_out, int parts, int r, float scaling, int rope_parts, int head_dim, int seq_len,
+                  float pos_scale, float base, void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 1 || K < 8 || K % 8 != 0 || n_out < 1 || parts < 1 || r < 0 || r > s2::kLoraMaxRank)
+    return S2ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return S2ATTN_ERR_INVALID_ARG;
+  if (r > 0 && (!aligned16(lora_a) || !lora_b || !std::isfinite(scaling))) return S2ATTN_ERR_INVALID_ARG;
+  if (rope_parts < 0 || rope_parts > parts) return S2ATTN_ERR_INVALID_ARG;
+  if (rope_parts > 0) {
+    if (head_dim != 32 && head_dim != 64 && head_dim != 128 && head_dim != 256) return S2ATTN_ERR_INVALID_ARG;
+    if (seq_len < 1 || T % seq_len != 0) return S2ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(pos_scale) || !std::isfinite(base) || !(base > 0.f)) return S2ATTN_ERR_INVALID_ARG;
+  }
+  if (n_out % s2::kLoraProjTileN != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if ((long long)parts * n_out > INT_MAX || (long long)T + 128 > INT_MAX) return S2ATTN_ERR_UNSUPPORTED;
+  if (((long long)T + 127) / 128 * ((long long)parts * n_out / s2::kLoraProjTileN) > INT_MAX)
+    return S2ATTN_ERR_UNSUPPORTED;
+  if (r > 0) {
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return S2ATTN_ERR_WORKSPACE;
+    if (workspace_bytes < lora_proj_workspace_bytes(T, K, n_out, parts, r)) return S2ATTN_ERR_WORKSPACE;
+  }
+  int* err = error_word_ptr();
+  if (!err) return S2ATTN_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return S2ATTN_ERR_CUDA;
+  RopeTable tab;
+  if (rope_parts > 0) {
+    int rc = rope_table(dev, seq_len, head_dim, pos_scale, base, &tab);
+    if (rc) return rc;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CUtensorMap tx, tw, tu, tb, ta;
+  if (!map_rows_bf16(&tx, x, 2, K, T, 1, 64, 128) ||
+      !map_rows_bf16(&tw, w, 2, K, (uint64_t)parts * n_out, 1, 64, s2::kLoraProjTileN))
+    return S2ATTN_ERR_CUDA;
+  tu = tx;
+  tb = tw;
+  if (r > 0) {
+    char* ws = static_cast<char*>(workspace);
+    void* u = ws;
+    void* a_pad = ws + lora_u_bytes(T, parts);
+    void* b_pad = ws + lora_u_bytes(T, parts) + align256((size_t)parts * s2::kLoraRankPad * K * 2);
+    if (!map_rows_bf16(&ta, a_pad, 2, K, (uint64_t)parts * s2::kLoraRankPad, 1, 64, s2::kLoraRankPad) ||
+        !map_rows_bf16(&tu, u, 3, s2::kLoraRankPad, T, parts, 64, 128) ||
+        !map_rows_bf16(&tb, b_pad, 2, s2::kLoraRankPad, (uint64_t)parts * n_out, 1, 64, s2::kLoraProjTileN))
+      return S2ATTN_ERR_CUDA;
+    cudaError_t e = s2::launch_lora_pad(lora_a, lora_b, a_pad, b_pad, parts, r, K, n_out, st);
+    if (e == cudaSuccess) e = s2::launch_lora_down(tx, ta, u, T, K, parts, scaling, sm_count(), err, st);
+    if (e != cudaSuccess) return S2ATTN_ERR_CUDA;
+  }
+  return cuda_status(s2::launch_lora_proj(tx, tw, tu, tb, y, T, K, n_out, parts, r, rope_parts, head_dim, seq_len,
+                                          tab.cos_d, tab.sin_d, sm_count(), err, st));
 }
 
 int s2attn_selftest_bounded_wait(unsigned timeout_us, void* stream) {

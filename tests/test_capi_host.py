@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     for required in ("s2attn_fwd", "s2attn_bwd", "rope_pi_apply", "s2attn_bwd_workspace_bytes",
                      "s2attn_fwd_f32", "s2attn_bwd_f32", "s2attn_get_device_error", "s2attn_decode",
-                     "s2attn_decode_workspace_bytes"):
+                     "s2attn_decode_workspace_bytes", "lora_proj_fwd", "lora_proj_workspace_bytes"):
         assert required in names
 
 
@@ -122,6 +122,50 @@ def test_workspace_checked_before_launch(lib):
     p = ctypes.c_void_p(0x10000)
     rc = lib.s2attn_bwd(p, p, p, p, p, p, p, p, p, 1, 1024, 2, 128, 512, 0, p, 16, NULL)
     assert rc == -3
+
+
+def test_lora_workspace_size(lib):
+    a256 = lambda n: (n + 255) // 256 * 256
+    # u [parts, T, 64] + a_pad [parts*64, K] + b_pad [parts*n_out, 64], bf16, each 256-aligned
+    assert lib.lora_proj_workspace_bytes(32768, 4096, 4096, 3, 8) == (
+        a256(3 * 32768 * 64 * 2) + a256(3 * 64 * 4096 * 2) + a256(3 * 4096 * 64 * 2))
+    assert lib.lora_proj_workspace_bytes(300, 520, 256, 3, 8) == a256(3 * 300 * 128) + a256(3 * 64 * 520 * 2) + 3 * 256 * 128
+    assert lib.lora_proj_workspace_bytes(300, 520, 256, 3, 0) == 0      # no adapter: no workspace
+    assert lib.lora_proj_workspace_bytes(300, 520, 256, 3, 65) == 0     # rank above 64: invalid
+    assert lib.lora_proj_workspace_bytes(0, 520, 256, 3, 8) == 0
+
+
+_P = 0x10000     # a 256-byte-aligned fake device address: these calls fail before any launch
+_WS = 1 << 26
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(K=12), -1),                                  # K % 8 != 0
+    (dict(K=0), -1),
+    (dict(r=65), -1),                                  # rank above 64
+    (dict(r=-1), -1),
+    (dict(parts=0), -1),
+    (dict(x=_P + 8), -1),                              # misaligned x
+    (dict(b=None), -1),                                # adapter without its up projection
+    (dict(scaling=float("nan")), -1),
+    (dict(rope_parts=4), -1),                          # more rotated parts than parts
+    (dict(rope_parts=2, head_dim=96), -1),             # head_dim outside {32, 64, 128, 256}
+    (dict(rope_parts=2, seq_len=7), -1),               # T not a multiple of seq_len
+    (dict(rope_parts=2, base=0.0), -1),
+    (dict(n_out=384), -2),                             # n_out not a multiple of the 256-column tile
+    (dict(ws_bytes=1024), -3),                         # workspace too small
+    (dict(ws=_P + 16), -3),                            # workspace not 256-byte aligned
+    (dict(ws=None), -3),
+])
+def test_lora_validation(lib, kw, status):
+    a = dict(x=_P, w=_P, a=_P, b=_P, y=_P, T=300, K=520, n_out=256, parts=3, r=8, scaling=2.0, rope_parts=0,
+             head_dim=128, seq_len=100, pos_scale=0.5, base=10000.0, ws=_P, ws_bytes=_WS)
+    a.update(kw)
+    vp = lambda v: None if v is None else ctypes.c_void_p(v)
+    rc = lib.lora_proj_fwd(vp(a["x"]), vp(a["w"]), vp(a["a"]), vp(a["b"]), vp(a["y"]), a["T"], a["K"], a["n_out"],
+                           a["parts"], a["r"], a["scaling"], a["rope_parts"], a["head_dim"], a["seq_len"],
+                           a["pos_scale"], a["base"], vp(a["ws"]), a["ws_bytes"], None)
+    assert rc == status
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):
