@@ -169,4 +169,4 @@ def rope_pi_bf16_at(x_bits, pos0, pos_scale, base=10000.0):
     return y
 
 
-from .lora import lora_proj  # noqa: E402  (numpy fp64; see lora.py)
+from .lora import lora_proj, lora_proj_bwd, rope_pi_bwd_f64  # noqa: E402  (numpy fp64; see lora.py)

@@ -100,3 +100,71 @@ def test_rejects_mismatched_shapes():
         oracle.lora_proj(x, w[:, :3], a, b, 1.0, 1)
     with pytest.raises(ValueError):
         oracle.lora_proj(x, w, a, b[:, :1], 1.0, 1)
+
+
+# ---- backward ------------------------------------------------------------------------
+
+def _loss(x, w, a, b, s, parts, dy):
+    """<y, dy>: its gradient with respect to any input is what lora_proj_bwd returns."""
+    return float((oracle.lora_proj(x, w, a, b, s, parts) * dy).sum())
+
+
+def test_backward_equals_central_finite_differences():
+    T, K, n_out, parts, r, s = 3, 5, 4, 2, 2, 1.25
+    x, w, a, b = _rand(11, T, K, n_out, parts, r)
+    dy = np.random.default_rng(12).standard_normal((parts, T, n_out))
+    dx, da, db = oracle.lora_proj_bwd(x, w, a, b, dy, s, parts)
+    h = 1e-6
+    for name, arr, grad in (("x", x, dx), ("a", a, da), ("b", b, db)):
+        num = np.empty_like(arr)
+        for idx in np.ndindex(arr.shape):
+            saved = arr[idx]
+            arr[idx] = saved + h
+            fp = _loss(x, w, a, b, s, parts, dy)
+            arr[idx] = saved - h
+            fm = _loss(x, w, a, b, s, parts, dy)
+            arr[idx] = saved
+            num[idx] = (fp - fm) / (2 * h)
+        rel = np.abs(num - grad).max() / np.abs(grad).max()
+        assert rel < 1e-7, (name, rel)
+
+
+def test_backward_hand_worked_example():
+    # the forward example above: x = [1, 2], W = [[3, 4], [5, 6]], A = [[1, -1]], B = [[2], [0.5]], s = 3
+    x = np.array([[1.0, 2.0]])
+    w = np.array([[3.0, 4.0], [5.0, 6.0]])
+    a = np.array([[1.0, -1.0]])
+    b = np.array([[2.0], [0.5]])
+    dy = np.array([[[1.0, -2.0]]])
+    dx, da, db = oracle.lora_proj_bwd(x, w, a, b, dy, 3.0, 1)
+    # dy B = 1*2 - 2*0.5 = 1;  dx = dy W + 3 * 1 * A = [3 - 10, 4 - 12] + [3, -3] = [-4, -11]
+    np.testing.assert_array_equal(dx, [[-4.0, -11.0]])
+    # dA = 3 * (dy B)^T x = 3 * [1, 2];  dB = 3 * dy^T (x A^T) = 3 * [1, -2]^T * (-1)
+    np.testing.assert_array_equal(da, [[3.0, 6.0]])
+    np.testing.assert_array_equal(db, [[-3.0], [6.0]])
+
+
+def test_backward_without_adapter_is_the_plain_linear_backward():
+    T, K, n_out, parts = 4, 6, 3, 3
+    x, w, _, _ = _rand(13, T, K, n_out, parts, 1)
+    dy = np.random.default_rng(14).standard_normal((parts, T, n_out))
+    dx, da, db = oracle.lora_proj_bwd(x, w, None, None, dy, 2.0, parts)
+    assert da is None and db is None
+    want = sum(dy[p] @ w[p * n_out:(p + 1) * n_out] for p in range(parts))
+    np.testing.assert_allclose(dx, want, rtol=1e-13, atol=1e-13)
+
+
+def test_rope_backward_undoes_the_forward_rotation():
+    """The rotation is orthogonal, so its transposed rotation (the backward) inverts the
+    C oracle's fp64 forward: rope_bwd(rope(y)) = y; and <rope(y), g> = <y, rope_bwd(g)>."""
+    rng = np.random.default_rng(15)
+    y = rng.standard_normal((2, 50, 3, 64))
+    g = rng.standard_normal(y.shape)
+    for ps in (1.0, 0.125):
+        np.testing.assert_allclose(oracle.rope_pi_bwd_f64(oracle.rope_pi_f64(y, ps), ps), y, rtol=0, atol=1e-12)
+        lhs = float((oracle.rope_pi_f64(y, ps) * g).sum())
+        rhs = float((y * oracle.rope_pi_bwd_f64(g, ps)).sum())
+        assert abs(lhs - rhs) <= 1e-10 * abs(lhs)
+    # position 0 is the identity
+    z = np.zeros((1, 1, 1, 8)); z[..., 3] = 1.0
+    np.testing.assert_array_equal(oracle.rope_pi_bwd_f64(z, 0.5), z)
