@@ -15,6 +15,11 @@ work of all ranks over the slowest rank's time ("scaling": "weak").
 
 --impl reference times the fp64 CPU oracle (the method's plain definition) on a
 bounded sample of the same workload, on this machine's host cores, rank 0 only.
+
+--mode sequence splits the workload's sequence across the ranks (whole groups per rank,
+the shifted heads' G/2 halo exchanged); --mode lora times the layer's LoRA-adapted
+projections (q/k/v with fused RoPE-PI, and o) alone.  The default run also reports the
+projections, the decoding step and full causal attention, outside the timed region.
 """
 import argparse
 import hashlib
@@ -577,6 +582,76 @@ def run_sequence_sharded(args, w):
     return 0
 
 
+def run_lora_projections(args, w):
+    """--mode lora: the LoRA-adapted projections of the workload's layer alone (one GPU; with
+    several ranks each runs the same calls and rank 0 reports), so that a profiler can capture
+    exactly these launches.  Five calls of lora_proj_fwd over T = B*N tokens, K = H*D: q, k, v
+    stacked with a rank-8 adapter and RoPE-PI fused on q and k; the same without RoPE; without
+    adapter or RoPE; o with the adapter; o without.  Each: `warmup` calls, then `steps` calls
+    timed with CUDA events.  value = the first one's TFLOP/s (2*T*K*outputs + adapter flops)."""
+    import torch
+
+    import shifted_sparse_attention_s2attn_b200 as s2
+
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    T, K, n, D = w.B * w.N, w.H * w.D, w.H * w.D, w.D
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(20)
+    x = torch.randn((T, K), generator=gen, device=dev).to(torch.bfloat16)
+    s2.clear_device_error()
+    out = {}
+    for name, parts, r, rope_parts in (("qkv_lora_rope", 3, 8, 2), ("qkv_lora", 3, 8, 0), ("qkv_plain", 3, 0, 0),
+                                       ("o_lora", 1, 8, 0), ("o_plain", 1, 0, 0)):
+        wt = (torch.randn((parts * n, K), generator=gen, device=dev) / K ** 0.5).to(torch.bfloat16)
+        a = (torch.randn((parts * r, K), generator=gen, device=dev) / K ** 0.5).to(torch.bfloat16) if r else None
+        b = (0.05 * torch.randn((parts * n, r), generator=gen, device=dev)).to(torch.bfloat16) if r else None
+        y = torch.empty((parts, T, n), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(256, s2.lora_proj_workspace_bytes(T, K, n, parts, r)), dtype=torch.uint8, device=dev)
+
+        def call():
+            s2.lora_proj_fwd(x, wt, a, b, y, parts, 2.0, rope_parts=rope_parts, head_dim=D, seq_len=w.N,
+                             pos_scale=w.pos_scale, workspace=ws, stream=stream)
+        for _ in range(args.warmup):
+            call()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / args.steps
+        flops = 2 * T * K * parts * n + 2 * T * K * parts * r + 2 * T * r * parts * n
+        out[name] = {"ms": ms, "tflops": flops / (ms / 1e3) / 1e12, "parts": parts, "r": r,
+                     "rope_parts": rope_parts}
+        del wt, a, b, y, ws
+    rc, detail = s2.get_device_error()
+    if rc != 0:
+        raise SystemExit(f"device error word set during the projection runs: {detail:#x}")
+    if rank != 0:
+        return 0
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    line = {"metric": "LoRA-adapted q/k/v projection with fused RoPE-PI, TFLOP/s", "value": out["qkv_lora_rope"]["tflops"],
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": out["qkv_lora_rope"]["ms"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "mode": "lora",
+            "config": {"workload": f"{w.name} layer projections: T={T} tokens, K={K}, q/k/v 3x{n} and o {n} "
+                                   f"outputs, LoRA rank 8, scaling 2, RoPE-PI pos_scale {w.pos_scale}"},
+            "roofline": {"kernel": "lora_gemm_kernel<256,true>", "bound": "tensor",
+                         "achieved": out["qkv_lora_rope"]["tflops"], "peak": peak, "unit": "TFLOP/s",
+                         "frac": out["qkv_lora_rope"]["tflops"] / peak, "traffic": None,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "note": "achieved covers the call's three kernels (pad, down projection, projection)"},
+            "calls": {k_: dict(v_, frac=v_["tflops"] / peak) for k_, v_ in out.items()},
+            "gpu_launches": sum(args.steps * (3 if v_["r"] else 1) for v_ in out.values())}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -585,9 +660,10 @@ def main():
     ap.add_argument("--workload", default="llama2_7b_32k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="replicas", choices=["replicas", "sequence"],
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "sequence", "lora"],
                     help="replicas: every rank runs the whole workload (default); sequence: the "
-                         "workload's sequence is split across the ranks")
+                         "workload's sequence is split across the ranks; lora: the layer's LoRA-adapted "
+                         "projections alone")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")
@@ -598,6 +674,8 @@ def main():
         return run_reference(args, w)
     if args.mode == "sequence":
         return run_sequence_sharded(args, w)
+    if args.mode == "lora":
+        return run_lora_projections(args, w)
     return run_ours(args, w)
 
 
