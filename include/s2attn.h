@@ -182,7 +182,9 @@ int rope_pi_apply_offset(void* q, void* k, int B, int N, int H, int D, int pos0,
  * the rotated parts are bit-identical to this call with rope_parts = 0 followed by
  * rope_pi_apply(y[p], ..., B, seq_len, n_out/head_dim, head_dim, pos_scale, base) on
  * each: the same table (cached per device, seq_len, head_dim, pos_scale, base) and the
- * same fp32 operation order, applied to the bf16-rounded projection.
+ * same fp32 operation order, applied to the bf16-rounded projection.  As for rope_pi_apply,
+ * the first call with a new table builds it on the host and copies it synchronously; make
+ * that call before any stream capture.
  * Requirements: K >= 8 and K % 8 == 0; 0 <= r <= 64; 0 <= rope_parts <= parts;
  * n_out % 256 == 0 (else S2ATTN_ERR_UNSUPPORTED); x, w, y, lora_a 16-byte aligned; with
  * rope_parts > 0: head_dim in {32, 64, 128, 256}, T % seq_len == 0, base > 0.
