@@ -98,9 +98,50 @@ def _bnhd(t, name):
     return tuple(t.shape)
 
 
+# The C entry points see only pointers, so the binding checks every tensor a call reads or
+# writes: first that each is contiguous with exactly the elements its role covers and the
+# expected dtype (_extent), then that all of them live on a CUDA device (_on_cuda).
+
+def _extent(t, name, numel, dtype):
+    if t is None or not t.is_contiguous() or t.numel() != numel or t.dtype != dtype:
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of {numel} elements")
+
+
+def _on_cuda(**tensors):
+    for name, t in tensors.items():
+        if t is not None and t.device.type != "cuda":
+            raise ValueError(f"{name} must be on a CUDA device")
+
+
+def _workspace(t):
+    if t is None or not t.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor")
+    _on_cuda(workspace=t)
+
+
+def _attn_args(dtype, shape, **tensors):
+    """Checks the [B,N,H,D] tensors (q's element count) and the [B,H,N] lse/delta of an
+    attention call (dq_acc: fp32 with q's element count), then their device."""
+    B, N, H, D = shape
+    for name, t in tensors.items():
+        if name in ("lse", "delta"):
+            _extent(t, name, B * H * N, _torch().float32)
+        elif name == "dq_acc":
+            _extent(t, name, B * N * H * D, _torch().float32)
+        else:
+            _extent(t, name, B * N * H * D, dtype)
+    _on_cuda(**tensors)
+
+
+def _torch():
+    import torch
+    return torch
+
+
 def s2attn_fwd(q, k, v, o, lse, G, shift_heads, stream=None):
     """bf16 forward: o <- S^2-Attn(q, k, v), lse <- [B,H,N] fp32 log-sum-exp."""
     B, N, H, D = _bnhd(q, "q")
+    _attn_args(_torch().bfloat16, (B, N, H, D), q=q, k=k, v=v, o=o, lse=lse)
     _check("s2attn_fwd", capi().s2attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, N, H, D, G,
                                            shift_heads, _stream(stream)))
 
@@ -113,6 +154,8 @@ def s2attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, workspace, str
     """bf16 backward into dq, dk, dv.  workspace: a uint8 device tensor of at least
     s2attn_bwd_workspace_bytes(B,N,H,D) bytes, 256-byte aligned."""
     B, N, H, D = _bnhd(q, "q")
+    _attn_args(_torch().bfloat16, (B, N, H, D), q=q, k=k, v=v, o=o, dout=dout, lse=lse, dq=dq, dk=dk, dv=dv)
+    _workspace(workspace)
     _check("s2attn_bwd", capi().s2attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
                                            _ptr(dk), _ptr(dv), B, N, H, D, G, shift_heads, _ptr(workspace),
                                            workspace.numel() * workspace.element_size(), _stream(stream)))
@@ -120,12 +163,15 @@ def s2attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, workspace, str
 
 def s2attn_bwd_preprocess(o, dout, delta, dq_acc, stream=None):
     B, N, H, D = _bnhd(o, "o")
+    _attn_args(_torch().bfloat16, (B, N, H, D), o=o, dout=dout, delta=delta, dq_acc=dq_acc)
     _check("s2attn_bwd_preprocess", capi().s2attn_bwd_preprocess(_ptr(o), _ptr(dout), _ptr(delta), _ptr(dq_acc),
                                                                  B, N, H, D, _stream(stream)))
 
 
 def s2attn_bwd_main(q, k, v, dout, lse, delta, dq_acc, dk, dv, G, shift_heads, stream=None):
     B, N, H, D = _bnhd(q, "q")
+    _attn_args(_torch().bfloat16, (B, N, H, D), q=q, k=k, v=v, dout=dout, lse=lse, delta=delta, dq_acc=dq_acc,
+               dk=dk, dv=dv)
     _check("s2attn_bwd_main", capi().s2attn_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(lse), _ptr(delta),
                                                      _ptr(dq_acc), _ptr(dk), _ptr(dv), B, N, H, D, G, shift_heads,
                                                      _stream(stream)))
@@ -133,6 +179,7 @@ def s2attn_bwd_main(q, k, v, dout, lse, delta, dq_acc, dk, dv, G, shift_heads, s
 
 def s2attn_bwd_dq_convert(dq_acc, dq, stream=None):
     B, N, H, D = _bnhd(dq, "dq")
+    _attn_args(_torch().bfloat16, (B, N, H, D), dq=dq, dq_acc=dq_acc)
     _check("s2attn_bwd_dq_convert", capi().s2attn_bwd_dq_convert(_ptr(dq_acc), _ptr(dq), B, N, H, D,
                                                                  _stream(stream)))
 
@@ -142,6 +189,7 @@ def s2attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, stream
     memory.  Uses the library's fixed device scratch (S2ATTN_NOALLOC_SCRATCH_BYTES per
     device, shared by all calls; overlapping calls race)."""
     B, N, H, D = _bnhd(q, "q")
+    _attn_args(_torch().bfloat16, (B, N, H, D), q=q, k=k, v=v, o=o, dout=dout, lse=lse, dq=dq, dk=dk, dv=dv)
     _check("s2attn_bwd_noalloc", capi().s2attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout),
                                                            _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, D, G,
                                                            shift_heads, _stream(stream)))
@@ -156,7 +204,17 @@ def s2attn_decode(q, k, v, o, lse, workspace, stream=None):
     against k, v [B,N,H,D]; o [B,M,H,D] bf16 and lse [B,H,M] fp32 are written.
     workspace: a uint8 device tensor of at least s2attn_decode_workspace_bytes bytes."""
     B, M, H, D = _bnhd(q, "q")
-    N = _bnhd(k, "k")[1]
+    Bk, N, Hk, Dk = _bnhd(k, "k")
+    if (Bk, Hk, Dk) != (B, H, D):
+        raise ValueError("k must be [B,N,H,D] with q's B, H and D")
+    bf16 = _torch().bfloat16
+    _extent(q, "q", B * M * H * D, bf16)
+    _extent(k, "k", B * N * H * D, bf16)
+    _extent(v, "v", B * N * H * D, bf16)
+    _extent(o, "o", B * M * H * D, bf16)
+    _extent(lse, "lse", B * H * M, _torch().float32)
+    _on_cuda(q=q, k=k, v=v, o=o, lse=lse)
+    _workspace(workspace)
     _check("s2attn_decode", capi().s2attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, M, N, H, D,
                                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
                                                  _stream(stream)))
@@ -164,12 +222,15 @@ def s2attn_decode(q, k, v, o, lse, workspace, stream=None):
 
 def s2attn_fwd_f32(q, k, v, o, lse, G, shift_heads, stream=None):
     B, N, H, D = _bnhd(q, "q")
+    _attn_args(_torch().float32, (B, N, H, D), q=q, k=k, v=v, o=o, lse=lse)
     _check("s2attn_fwd_f32", capi().s2attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, N, H, D, G,
                                                    shift_heads, _stream(stream)))
 
 
 def s2attn_bwd_f32(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, workspace, stream=None):
     B, N, H, D = _bnhd(q, "q")
+    _attn_args(_torch().float32, (B, N, H, D), q=q, k=k, v=v, o=o, dout=dout, lse=lse, dq=dq, dk=dk, dv=dv)
+    _workspace(workspace)
     _check("s2attn_bwd_f32", capi().s2attn_bwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
                                                    _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, D, G, shift_heads,
                                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -180,6 +241,10 @@ def rope_pi_apply(q, k, pos_scale, base=10000.0, stream=None):
     """In-place RoPE with position interpolation on bf16 q and/or k ([B,N,H,D])."""
     ref = q if q is not None else k
     B, N, H, D = _bnhd(ref, "q/k")
+    for name, t in (("q", q), ("k", k)):
+        if t is not None:
+            _extent(t, name, B * N * H * D, _torch().bfloat16)
+    _on_cuda(q=q, k=k)
     _check("rope_pi_apply", capi().rope_pi_apply(_ptr(q), _ptr(k), B, N, H, D, float(pos_scale), float(base),
                                                  _stream(stream)))
 
@@ -188,6 +253,10 @@ def rope_pi_apply_offset(q, k, pos0, pos_scale, base=10000.0, stream=None):
     """In-place RoPE-PI on bf16 q and/or k whose row t is the token at position pos0 + t."""
     ref = q if q is not None else k
     B, N, H, D = _bnhd(ref, "q/k")
+    for name, t in (("q", q), ("k", k)):
+        if t is not None:
+            _extent(t, name, B * N * H * D, _torch().bfloat16)
+    _on_cuda(q=q, k=k)
     _check("rope_pi_apply_offset", capi().rope_pi_apply_offset(_ptr(q), _ptr(k), B, N, H, D, int(pos0),
                                                                float(pos_scale), float(base), _stream(stream)))
 
@@ -203,15 +272,34 @@ def lora_proj_fwd(x, w, lora_a, lora_b, y, parts, scaling, rope_parts=0, head_di
     [parts*r, K] and lora_b: [parts*n_out, r] (both None for r = 0), y: [parts, T, n_out]
     (or any contiguous tensor of that many elements); all bf16 on the device.  workspace:
     uint8 device tensor of lora_proj_workspace_bytes(T, K, n_out, parts, r) bytes (r > 0)."""
+    import torch
+    if (lora_a is None) != (lora_b is None):
+        raise ValueError("lora_a and lora_b are given together (or both None for no adapter)")
     for t, name in ((x, "x"), (w, "w"), (y, "y"), (lora_a, "lora_a"), (lora_b, "lora_b")):
-        if t is not None and not t.is_contiguous():
+        if t is None:
+            continue
+        if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be bf16")
+    # The C entry point sees only pointers: every extent it will read or write is checked here.
     K = x.shape[-1]
     T = x.numel() // K
+    if parts < 1 or w.dim() != 2 or w.shape[1] != K or w.shape[0] % parts:
+        raise ValueError("w must be [parts*n_out, K] with x's K")
     n_out = w.shape[0] // parts
-    r = 0 if lora_a is None else lora_a.shape[0] // parts
+    r = 0
+    if lora_a is not None:
+        if lora_a.dim() != 2 or lora_a.shape[1] != K or lora_a.shape[0] % parts:
+            raise ValueError("lora_a must be [parts*r, K]")
+        r = lora_a.shape[0] // parts
+        if tuple(lora_b.shape) != (parts * n_out, r):
+            raise ValueError("lora_b must be [parts*n_out, r]")
     if y.numel() != parts * T * n_out:
         raise ValueError("y must hold parts * T * n_out elements")
+    _on_cuda(x=x, w=w, y=y, lora_a=lora_a, lora_b=lora_b)
+    if r > 0:
+        _workspace(workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("lora_proj_fwd", capi().lora_proj_fwd(
         _ptr(x), _ptr(w), _ptr(lora_a), _ptr(lora_b), _ptr(y), T, K, n_out, parts, r, float(scaling),

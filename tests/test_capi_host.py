@@ -201,3 +201,28 @@ def test_debug_build_exports_the_same_boundary(lib):
     for name in _declared_functions():
         assert hasattr(debug, name), name
     assert debug.s2attn_version() == 100
+
+
+def test_lora_binding_checks_extents_before_the_call(lib):
+    """The C entry point sees only pointers; the binding rejects tensors whose extents do not
+    match before anything is passed on (CPU tensors suffice: nothing reaches the library)."""
+    import torch
+    import shifted_sparse_attention_s2attn_b200 as s2
+    bf = dict(dtype=torch.bfloat16)
+    x, w = torch.zeros(300, 520, **bf), torch.zeros(3 * 256, 520, **bf)
+    a, b = torch.zeros(3 * 8, 520, **bf), torch.zeros(3 * 256, 8, **bf)
+    y = torch.zeros(3, 300, 256, **bf)
+    bad = [
+        dict(w=torch.zeros(3 * 256, 512, **bf)),         # K differs from x's
+        dict(w=torch.zeros(3 * 256 + 1, 520, **bf)),     # rows not a multiple of parts
+        dict(a=torch.zeros(3 * 8, 512, **bf)),           # adapter K differs
+        dict(b=torch.zeros(3 * 256, 4, **bf)),           # rank differs between A and B
+        dict(b=None),                                    # A without B
+        dict(y=torch.zeros(3, 299, 256, **bf)),          # output too small
+        dict(x=torch.zeros(300, 520)),                   # fp32, not bf16
+    ]
+    for kw in bad:
+        args = dict(x=x, w=w, a=a, b=b, y=y)
+        args.update(kw)
+        with pytest.raises(ValueError):
+            s2.lora_proj_fwd(args["x"], args["w"], args["a"], args["b"], args["y"], 3, 2.0)

@@ -147,8 +147,9 @@ def test_bf16_rejects_unsupported_shapes():
         s2.s2attn_fwd(q, q, q, o, lse, 96, 0)       # G not a multiple of 128
     assert e.value.status == -2
     q64 = torch.zeros((1, 256, 2, 64), dtype=torch.bfloat16, device="cuda")
+    lse64 = torch.empty((1, 2, 256), dtype=torch.float32, device="cuda")
     with pytest.raises(s2.S2AttnError) as e:
-        s2.s2attn_fwd(q64, q64, q64, torch.empty_like(q64), lse, 128, 0)   # D = 64: fp32 path only
+        s2.s2attn_fwd(q64, q64, q64, torch.empty_like(q64), lse64, 128, 0)   # D = 64: fp32 path only
     assert e.value.status == -2
 
 
