@@ -148,6 +148,9 @@ int s2attn_bwd_f32(const float* q, const float* k, const float* v, const float* 
  * The cos/sin table is computed on the host on first use of each (device, N, D,
  * pos_scale, base) and cached in device memory owned by the library until exit.
  * Either q or k may be NULL.  Requires D % 16 == 0, D <= 256.
+ * Backward: with -pos_scale every angle is negated exactly (the products above round
+ * symmetrically, cos is even and sin odd), which applies the transposed rotation -- the
+ * gradient through RoPE-PI -- to dq and dk in the same operation order.
  */
 int rope_pi_apply(void* q, void* k, int B, int N, int H, int D, float pos_scale, float base, void* stream);
 

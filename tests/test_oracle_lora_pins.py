@@ -168,3 +168,29 @@ def test_rope_backward_undoes_the_forward_rotation():
     # position 0 is the identity
     z = np.zeros((1, 1, 1, 8)); z[..., 3] = 1.0
     np.testing.assert_array_equal(oracle.rope_pi_bwd_f64(z, 0.5), z)
+
+
+def test_rope_backward_is_rope_with_negated_pos_scale():
+    """Rotating by -a is the transposed rotation, and every step of the fp32 evaluation order
+    flips sign exactly when pos_scale does (t * ps and (t * ps) * theta round symmetrically,
+    cos is even, sin is odd), so RoPE-PI with -pos_scale is the RoPE backward: in fp64 equal to
+    rope_pi_bwd_f64, and in the bit-exact fp32 order within one bf16 rounding of it."""
+    import math
+    from shifted_sparse_attention_s2attn_b200.synthetic import f32_to_bf16_bits
+    rng = np.random.default_rng(16)
+    g = rng.standard_normal((1, 300, 2, 128))
+    for ps in (1.0, 0.125, 0.04):
+        np.testing.assert_allclose(oracle.rope_pi_f64(g, -ps), oracle.rope_pi_bwd_f64(g, ps), rtol=0, atol=1e-12)
+        bits = f32_to_bf16_bits(g.astype(np.float32))
+        inv = bf16_bits_to_f32(oracle.rope_pi_bf16(bits, -ps)).astype(np.float64)
+        ref = oracle.rope_pi_bwd_f64(bf16_bits_to_f32(bits).astype(np.float64), ps)
+        # bf16 rounding of each output, plus the fp32 angle's rounding (half an fp32 ulp of angles
+        # up to 300 rad here, ~1.5e-5 rad) times the pair's size
+        err = np.abs(inv - ref)
+        assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 2.0 ** -12 * np.abs(g).max())
+        assert np.abs(inv - bf16_bits_to_f32(oracle.rope_pi_bf16(bits, ps)).astype(np.float64)).max() > 0.5
+    # the host libm the tables are built with: (float) cos / sin of +-a in double, over many a
+    for a in np.linspace(-5000.0, 5000.0, 20011):
+        a32 = float(np.float32(a))
+        assert np.float32(math.cos(-a32)) == np.float32(math.cos(a32))
+        assert np.float32(math.sin(-a32)) == -np.float32(math.sin(a32))
