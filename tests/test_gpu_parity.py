@@ -46,6 +46,30 @@ def test_rope_pi_bit_exact(B, N, H, D, scale):
     np.testing.assert_array_equal(device_to_bits(k), oracle.rope_pi_bf16(k_bits, scale))
 
 
+@pytest.mark.parametrize("N,H,D,scale", [(512, 4, 128, 0.5), (32768, 2, 128, 1 / 8)])
+def test_rope_backward_is_rope_with_negated_scale(N, H, D, scale):
+    """The gradient through RoPE-PI (the transposed rotation) is rope_pi_apply with -pos_scale:
+    bit-exact to the fp32-order oracle at -pos_scale, and the forward followed by it returns the
+    input to within two bf16 roundings of the pair's size (doubled)."""
+    from parity_utils import bits_to_device
+    g_bits = _bits((1, N, H, D), 3)
+    g = bits_to_device(g_bits)
+    s2.rope_pi_apply(g, None, -scale)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(device_to_bits(g), oracle.rope_pi_bf16(g_bits, -scale))
+    y = bits_to_device(g_bits)
+    s2.rope_pi_apply(y, None, scale)
+    s2.rope_pi_apply(y, None, -scale)
+    torch.cuda.synchronize()
+    x = bf16_bits_to_f32(g_bits).astype(np.float64)
+    back = y.float().cpu().numpy().astype(np.float64)
+    # each bf16 rounding is at most 2^-8 of a rotated element, which is at most |x1| + |x2| of its pair
+    half = D // 2
+    pair = np.abs(x[..., :half]) + np.abs(x[..., half:])
+    pair = np.concatenate([pair, pair], axis=-1)
+    assert np.all(np.abs(back - x) <= 2.0 ** -6 * pair + 2.0 ** -20)
+
+
 def test_rope_pi_k_only_and_repeat():
     from parity_utils import bits_to_device
     k_bits = _bits((1, 256, 2, 128), 3)
