@@ -189,7 +189,7 @@ int rope_pi_apply_offset(void* q, void* k, int B, int N, int H, int D, int pos0,
  * the first call with a new table builds it on the host and copies it synchronously; make
  * that call before any stream capture.
  * Requirements: K >= 8 and K % 8 == 0; 0 <= r <= 64; 0 <= rope_parts <= parts;
- * n_out % 256 == 0 (else S2ATTN_ERR_UNSUPPORTED); x, w, y, lora_a 16-byte aligned; with
+ * n_out % 256 == 0 and K >= 64 (else S2ATTN_ERR_UNSUPPORTED); x, w, y, lora_a 16-byte aligned; with
  * rope_parts > 0: head_dim in {32, 64, 128, 256}, T % seq_len == 0, base > 0.
  * `workspace` (device, caller-owned, 256-byte aligned, at least
  * lora_proj_workspace_bytes(T, K, n_out, parts, r) bytes; may be NULL when r == 0) holds the

@@ -445,6 +445,7 @@ int lora_proj_fwd(const void* x, const void* w, const void* lora_a, const void* 
     if (!std::isfinite(pos_scale) || !std::isfinite(base) || !(base > 0.f)) return S2ATTN_ERR_INVALID_ARG;
   }
   if (n_out % s2::kLoraProjTileN != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if (K < 64) return S2ATTN_ERR_UNSUPPORTED;   // the tensor maps' 64-column boxes must fit in a row of x and W
   if ((long long)parts * n_out > INT_MAX || (long long)T + 128 > INT_MAX) return S2ATTN_ERR_UNSUPPORTED;
   if (((long long)T + 127) / 128 * ((long long)parts * n_out / s2::kLoraProjTileN) > INT_MAX)
     return S2ATTN_ERR_UNSUPPORTED;

@@ -153,6 +153,7 @@ _WS = 1 << 26
     (dict(rope_parts=2, seq_len=7), -1),               # T not a multiple of seq_len
     (dict(rope_parts=2, base=0.0), -1),
     (dict(n_out=384), -2),                             # n_out not a multiple of the 256-column tile
+    (dict(K=56), -2),                                  # K below one 64-column box
     (dict(ws_bytes=1024), -3),                         # workspace too small
     (dict(ws=_P + 16), -3),                            # workspace not 256-byte aligned
     (dict(ws=None), -3),
