@@ -188,11 +188,20 @@ def _sample_units(w):
 
 
 def _sample_rows(G, seed):
+    """Query rows and key rows (rolled-local) of one group.  The key rows cover the whole walk
+    of the backward: key tile 0 (seen by every query tile of the group: the longest dK/dV
+    accumulation), the tile starting at G/2 (the wrap point of a shifted head's roll) and the
+    one before it, a random middle tile, and the last two tiles (seen by one or two query tiles)."""
     rng = np.random.default_rng(seed)
     qrows = sorted({0, 1, 63, 64, 127, 128, 129, G // 2 - 1, G // 2, G - 129, G - 128, G - 2, G - 1,
                     *rng.integers(0, G, 6).tolist()})
-    krows = sorted({G - 1, G - 2, G - 64, G - 65, G - 127, G - 128, *rng.integers(G - 256, G, 4).tolist()})
-    return qrows, krows
+    n_kt = G // 128
+    mid = int(rng.integers(1, max(2, n_kt - 1))) * 128
+    krows = sorted({0, 1, 2, 63, 64, 126, 127,                      # key tile 0
+                    G // 2 - 1, G // 2, G // 2 + 1, G // 2 + 127,   # around the wrap point
+                    mid, mid + 1 + int(rng.integers(0, 126)),       # a middle tile
+                    G - 1, G - 2, G - 64, G - 65, G - 127, G - 128, *rng.integers(G - 256, G, 4).tolist()})
+    return qrows, [r for r in krows if 0 <= r < G]
 
 
 @pytest.mark.parametrize("wname", ["llama2_7b_8k", "llama2_7b_32k", "llama2_7b_32k_full_causal",
@@ -211,6 +220,7 @@ def test_bf16_full_size_sampled(wname):
     worst = {"o": 0.0, "lse": 0.0}
     got_g = {g: [] for g in ("dq", "dk", "dv")}
     ref_g = {g: [] for g in ("dq", "dk", "dv")}
+    got_t0, ref_t0 = {"dk": [], "dv": []}, {"dk": [], "dv": []}
     for (b, h, j) in _sample_units(w):
         qrows, krows = _sample_rows(w.G, 1000 * h + j)
         r = oracle.s2attn_unit(q_bits, k_bits, inp["v"], w.G, w.shift_heads, b, h, j, qrows=qrows,
@@ -224,12 +234,19 @@ def test_bf16_full_size_sampled(wname):
             got_g["dq"].append(out["dq"][b, qt, h].float().cpu().numpy()); ref_g["dq"].append(r["dq"])
             got_g["dk"].append(out["dk"][b, kt, h].float().cpu().numpy()); ref_g["dk"].append(r["dk"])
             got_g["dv"].append(out["dv"][b, kt, h].float().cpu().numpy()); ref_g["dv"].append(r["dv"])
+            # key tile 0 alone: the longest accumulation must not hide behind the short ones
+            t0 = np.asarray(krows) < 128
+            got_t0["dk"].append(got_g["dk"][-1][t0]); ref_t0["dk"].append(r["dk"][t0])
+            got_t0["dv"].append(got_g["dv"][-1][t0]); ref_t0["dv"].append(r["dv"][t0])
     assert worst["o"] <= TOL_O_BF16, (wname, worst)
     assert worst["lse"] <= TOL_LSE_BF16, (wname, worst)
     if bwd:
         for g in ("dq", "dk", "dv"):
             e = rel_l2(np.concatenate(got_g[g]), np.concatenate(ref_g[g]))
             assert e <= TOL_REL_L2_BF16, (wname, g, e)
+        for g in ("dk", "dv"):
+            e = rel_l2(np.concatenate(got_t0[g]), np.concatenate(ref_t0[g]))
+            assert e <= TOL_REL_L2_BF16, (wname, g, "key tile 0", e)
     # properties that hold at any size, over the whole output
     assert torch.isfinite(out["o"]).all() and torch.isfinite(out["lse"]).all()
     if bwd:
