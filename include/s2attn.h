@@ -211,12 +211,16 @@ int lora_proj_fwd(const void* x, const void* w, const void* lora_a, const void* 
  * s2attn_bwd a workspace.
  * Same arguments, shape rules and results as s2attn_bwd, minus the workspace: the
  * fp32 dQ accumulator and delta live in a fixed array of
- * S2ATTN_NOALLOC_SCRATCH_BYTES in the library's device memory, reserved on every
- * device where the library's module is loaded and held until the process exits.
+ * S2ATTN_NOALLOC_SCRATCH_BYTES in the library's device memory, held until the
+ * process exits.  The array is reserved when the module holding it is loaded on a
+ * device; with CUDA's lazy module loading (the default) that happens inside the
+ * first call on each device, which looks up the array's device address (with that
+ * device current) and caches it.  So the first call on a device does take
+ * S2ATTN_NOALLOC_SCRATCH_BYTES of device memory: make it before the caller's own
+ * allocator reserves the device (else it fails with S2ATTN_ERR_CUDA) and before any
+ * stream capture.  Later calls take no device memory.
  * Problems needing more (B*N*H*D*4 + B*H*N*4 bytes, each part rounded up to 256)
  * return S2ATTN_ERR_WORKSPACE; at D = 128 that is about 130k (token, head) rows.
- * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream capture.
  * Every call uses the same array and leaves its last contents there (the
  * accumulator is zeroed at the start of each call): calls whose work overlaps on
  * the GPU -- on different streams, or on different host threads -- race on it.

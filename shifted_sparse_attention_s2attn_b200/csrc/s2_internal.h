@@ -12,6 +12,10 @@ namespace s2 {
 // code = (kernel << 8) | site
 enum Kernel : int { K_FWD = 1, K_BWD = 2, K_SELFTEST = 3, K_DEC = 4, K_LORA = 5 };
 
+// Argument rules of the bf16 tensor-core entry points (shape, D == 128, tile alignment of G and
+// G/2, and the index-overflow guards): S2ATTN_OK or the status those entry points return.
+int check_tensor_core_args(int B, int N, int H, int D, int G, int shift_heads);
+
 // Problem description after validation.  Rows of a [B,N,H,D] tensor for head h
 // are addressed through 3-D tensor maps with dims {D, H, B*N}.
 struct Shape {

@@ -230,6 +230,12 @@ size_t decode_part_o_bytes(int B, int M, int N, int H, int D) {
 
 }  // namespace
 
+namespace s2 {
+int check_tensor_core_args(int B, int N, int H, int D, int G, int shift_heads) {
+  return check_tensor_core_shape(B, N, H, D, G, shift_heads);
+}
+}  // namespace s2
+
 extern "C" {
 
 int s2attn_version(void) { return 100; }

@@ -15,8 +15,10 @@
 
 namespace {
 
-// The scratch: S2ATTN_NOALLOC_SCRATCH_BYTES per device, reserved when this module is
-// loaded on a device and held until the process exits.  Every call shares it.
+// The scratch: S2ATTN_NOALLOC_SCRATCH_BYTES per device, reserved when this file's module is
+// loaded on a device and held until the process exits.  Every call shares it.  Under CUDA's
+// lazy module loading (the default) the module is loaded by the first address lookup below,
+// i.e. inside the first call on each device: that call is where the memory is taken.
 static __device__ __align__(256) unsigned char g_bwd_scratch[S2ATTN_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -45,20 +47,17 @@ void* scratch_ptr() {
 extern "C" int s2attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
                                   const float* lse, void* dq, void* dk, void* dv, int B, int N, int H, int D, int G,
                                   int shift_heads, void* stream) {
-  // Argument rules of s2attn_bwd, checked here so that nothing is enqueued on error.
-  if (B < 1 || N < 1 || H < 1 || D < 1 || G < 1 || N % G != 0 || shift_heads < 0 || shift_heads > H ||
-      (shift_heads > 0 && G % 2 != 0))
-    return S2ATTN_ERR_INVALID_ARG;
-  if (D != 128 || G % 128 != 0 || (shift_heads > 0 && (G / 2) % 128 != 0)) return S2ATTN_ERR_UNSUPPORTED;
+  // The argument rules of s2attn_bwd (the same check, overflow guards included), applied
+  // here so that nothing is enqueued on error.
+  int rc = s2::check_tensor_core_args(B, N, H, D, G, shift_heads);
+  if (rc) return rc;
   const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv};
   for (const void* ptr : ptrs)
     if (!ptr || (reinterpret_cast<uintptr_t>(ptr) & 15u)) return S2ATTN_ERR_INVALID_ARG;
   const size_t elems = (size_t)B * N * H * D;
-  if (elems > (size_t)S2ATTN_NOALLOC_SCRATCH_BYTES) return S2ATTN_ERR_WORKSPACE;
   const size_t acc_bytes = align256(elems * sizeof(float));
   if (acc_bytes + align256((size_t)B * H * N * sizeof(float)) > (size_t)S2ATTN_NOALLOC_SCRATCH_BYTES)
     return S2ATTN_ERR_WORKSPACE;  // the problem does not fit the fixed scratch
-  int rc;
   char* base = static_cast<char*>(scratch_ptr());
   if (!base) return S2ATTN_ERR_CUDA;
   float* dq_acc = reinterpret_cast<float*>(base);
