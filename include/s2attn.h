@@ -125,6 +125,32 @@ int s2attn_decode(const void* q, const void* k, const void* v, void* o, float* l
                   int D, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Halo rows of sequence-sharded S^2-Attn.  The groups are independent, so a sequence
+ * split across ranks in whole groups needs one exchange ("LongLoRA paper notes",
+ * section 3.3; nearauto.com article, "shift short attention" steps (1) and (2)).  A
+ * rank holding tokens [t0, t0+N) of every head (N a multiple of G) runs the forward and
+ * backward above on its own tensors with the shift; their last rolled group of a
+ * shifted head reads the rank's tail and then its rows [0, G/2).  Those rows of the
+ * shifted heads belong to the previous rank's last group, so the sharded path swaps the
+ * next rank's first G/2 rows (the halo) into them for the duration of the calls and
+ * swaps them back afterwards; the results written to them belong to the halo's tokens
+ * and are returned to their owner.  These two calls are the copies that swap needs:
+ *   s2attn_halo_rows: for each of n_tensors bf16 [B,N,H,D] tensors x[i] and contiguous
+ *     buffers buf[i] [B, G/2, shift_heads, D]:  to_buf != 0: buf[i][b,r,s,:] =
+ *     x[i][b, r, H-shift_heads+s, :] for r < G/2;  to_buf == 0: the reverse copy.
+ *   s2attn_halo_lse: the same rows of fp32 [B,H,N] tensors (lse, softmax statistics),
+ *     buffers [B, shift_heads, G/2].
+ * x and buf are host arrays of n_tensors device pointers (1 <= n_tensors <= 8), bf16
+ * pointers 16-byte aligned (lse pointers 4-byte aligned), owned by the caller.
+ * Requirements: G divides N, G even, 1 <= shift_heads <= H, D*2 a multiple of 16.
+ * One kernel launch per call on `stream`; buffers and tensors must not overlap.
+ */
+int s2attn_halo_rows(void* const* x, void* const* buf, int n_tensors, int to_buf, int B, int N, int H, int D,
+                     int G, int shift_heads, void* stream);
+int s2attn_halo_lse(float* const* lse, float* const* buf, int n_tensors, int to_buf, int B, int N, int H, int G,
+                    int shift_heads, void* stream);
+
+/*
  * fp32 forward/backward on CUDA cores, any valid shape with 1 <= D <= 128
  * (G >= 1 divides N; G even when shift_heads > 0).  Same tensor layouts, all fp32.
  * s2attn_bwd_f32 uses the delta part of the workspace only
@@ -201,6 +227,24 @@ size_t lora_proj_workspace_bytes(int T, int K, int n_out, int parts, int r);
 int lora_proj_fwd(const void* x, const void* w, const void* lora_a, const void* lora_b, void* y, int T, int K,
                   int n_out, int parts, int r, float scaling, int rope_parts, int head_dim, int seq_len,
                   float pos_scale, float base, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward of lora_proj_fwd for training (the frozen W gets no gradient; notes section 3.2):
+ *   dx       = sum_p dy_p W_p + s (dy_p B_p) A_p           [T, K]
+ *   d_lora_a = per part, s (dy_p B_p)^T x                  [parts*r, K]
+ *   d_lora_b = per part, s dy_p^T (x A_p^T)                [parts*n_out, r]
+ * dy [parts, T, n_out] is the gradient of y before RoPE: take dq and dk back through the
+ * rotation first with rope_pi_apply(dq, dk, ..., -pos_scale, ...).  Same layouts and
+ * requirements as lora_proj_fwd (K >= 64, n_out % 256 == 0, r <= 64); d_lora_a / d_lora_b may be
+ * NULL when r == 0.  `workspace` (device, caller-owned, 256-byte aligned, at least
+ * lora_proj_bwd_workspace_bytes bytes) holds the padded adapters, the recomputed intermediate
+ * s x A^T, s dy B, and fp32 accumulators for the adapter gradients.  The adapter gradients add
+ * fp32 partial sums over token ranges, so they are not bitwise reproducible run to run.
+ */
+size_t lora_proj_bwd_workspace_bytes(int T, int K, int n_out, int parts, int r);
+int lora_proj_bwd(const void* x, const void* w, const void* lora_a, const void* lora_b, const void* dy, void* dx,
+                  void* d_lora_a, void* d_lora_b, int T, int K, int n_out, int parts, int r, float scaling,
+                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Backward pass that allocates nothing.  The LongLoRA pages have no counterpart of

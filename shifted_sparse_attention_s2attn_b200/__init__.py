@@ -13,7 +13,8 @@ __all__ = [
     "S2AttnError", "capi", "library_path",
     "s2attn_fwd", "s2attn_bwd", "s2attn_bwd_workspace_bytes", "s2attn_bwd_preprocess", "s2attn_bwd_main",
     "s2attn_bwd_dq_convert", "s2attn_bwd_noalloc", "s2attn_decode", "s2attn_decode_workspace_bytes", "s2attn_fwd_f32", "s2attn_bwd_f32", "rope_pi_apply", "rope_pi_apply_offset",
-    "lora_proj_fwd", "lora_proj_workspace_bytes",
+    "lora_proj_fwd", "lora_proj_workspace_bytes", "lora_proj_bwd", "lora_proj_bwd_workspace_bytes",
+    "s2attn_halo_rows", "s2attn_halo_lse",
     "get_device_error", "clear_device_error", "s2attn_selftest_bounded_wait",
 ]
 
@@ -62,6 +63,10 @@ def capi():
         "rope_pi_apply_offset": ([P, P, I, I, I, I, I, F, F, P], I),
         "lora_proj_workspace_bytes": ([I, I, I, I, I], Z),
         "lora_proj_fwd": ([P, P, P, P, P, I, I, I, I, I, F, I, I, I, F, F, P, Z, P], I),
+        "lora_proj_bwd_workspace_bytes": ([I, I, I, I, I], Z),
+        "lora_proj_bwd": ([P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, Z, P], I),
+        "s2attn_halo_rows": ([ctypes.POINTER(P), ctypes.POINTER(P), I, I, I, I, I, I, I, I, P], I),
+        "s2attn_halo_lse": ([ctypes.POINTER(P), ctypes.POINTER(P), I, I, I, I, I, I, I, P], I),
         "s2attn_get_device_error": ([ctypes.POINTER(I)], I),
         "s2attn_clear_device_error": ([], I),
         "s2attn_selftest_bounded_wait": ([ctypes.c_uint, P], I),
@@ -195,6 +200,42 @@ def s2attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, stream
                                                            shift_heads, _stream(stream)))
 
 
+def _ptr_array(ts):
+    return (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+
+
+def s2attn_halo_rows(xs, bufs, to_buf, G, shift_heads, stream=None):
+    """Rows [0, G/2) of the shifted heads of each bf16 [B,N,H,D] tensor in xs to (to_buf=True)
+    or from (False) the matching contiguous [B, G/2, shift_heads, D] buffer in bufs; one launch."""
+    if not xs or len(xs) != len(bufs):
+        raise ValueError("xs and bufs must be non-empty lists of equal length")
+    B, N, H, D = _bnhd(xs[0], "x")
+    bf16 = _torch().bfloat16
+    for i, (x, b) in enumerate(zip(xs, bufs)):
+        _extent(x, f"x[{i}]", B * N * H * D, bf16)
+        _extent(b, f"buf[{i}]", B * (G // 2) * shift_heads * D, bf16)
+        _on_cuda(x=x, buf=b)
+    _check("s2attn_halo_rows", capi().s2attn_halo_rows(_ptr_array(xs), _ptr_array(bufs), len(xs), int(bool(to_buf)),
+                                                       B, N, H, D, G, shift_heads, _stream(stream)))
+
+
+def s2attn_halo_lse(lses, bufs, to_buf, G, shift_heads, stream=None):
+    """The same rows of fp32 [B,H,N] tensors (softmax statistics) to or from [B, shift_heads, G/2]
+    buffers; one launch."""
+    if not lses or len(lses) != len(bufs):
+        raise ValueError("lses and bufs must be non-empty lists of equal length")
+    if lses[0].dim() != 3:
+        raise ValueError("lse must be a [B,H,N] tensor")
+    B, H, N = tuple(lses[0].shape)
+    f32 = _torch().float32
+    for i, (x, b) in enumerate(zip(lses, bufs)):
+        _extent(x, f"lse[{i}]", B * H * N, f32)
+        _extent(b, f"buf[{i}]", B * shift_heads * (G // 2), f32)
+        _on_cuda(lse=x, buf=b)
+    _check("s2attn_halo_lse", capi().s2attn_halo_lse(_ptr_array(lses), _ptr_array(bufs), len(lses),
+                                                     int(bool(to_buf)), B, N, H, G, shift_heads, _stream(stream)))
+
+
 def s2attn_decode_workspace_bytes(B, M, N, H, D):
     return int(capi().s2attn_decode_workspace_bytes(B, M, N, H, D))
 
@@ -305,6 +346,39 @@ def lora_proj_fwd(x, w, lora_a, lora_b, y, parts, scaling, rope_parts=0, head_di
         _ptr(x), _ptr(w), _ptr(lora_a), _ptr(lora_b), _ptr(y), T, K, n_out, parts, r, float(scaling),
         int(rope_parts), int(head_dim), int(seq_len if seq_len is not None else T), float(pos_scale), float(base),
         _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def lora_proj_bwd_workspace_bytes(T, K, n_out, parts, r):
+    return int(capi().lora_proj_bwd_workspace_bytes(T, K, n_out, parts, r))
+
+
+def lora_proj_bwd(x, w, lora_a, lora_b, dy, dx, d_lora_a, d_lora_b, parts, scaling, workspace, stream=None):
+    """Backward of lora_proj_fwd (W frozen): dx [T, K], d_lora_a [parts*r, K], d_lora_b
+    [parts*n_out, r] from dy [parts, T, n_out] (the gradient before RoPE; rope_pi_apply with
+    -pos_scale takes dq, dk back through it)."""
+    torch = _torch()
+    K = x.shape[-1]
+    T = x.numel() // K
+    if parts < 1 or w.dim() != 2 or w.shape[1] != K or w.shape[0] % parts:
+        raise ValueError("w must be [parts*n_out, K] with x's K")
+    n_out = w.shape[0] // parts
+    r = 0 if lora_a is None else lora_a.shape[0] // parts
+    bf = torch.bfloat16
+    _extent(x, "x", T * K, bf)
+    _extent(w, "w", parts * n_out * K, bf)
+    _extent(dy, "dy", parts * T * n_out, bf)
+    _extent(dx, "dx", T * K, bf)
+    if r:
+        _extent(lora_a, "lora_a", parts * r * K, bf)
+        _extent(lora_b, "lora_b", parts * n_out * r, bf)
+        _extent(d_lora_a, "d_lora_a", parts * r * K, bf)
+        _extent(d_lora_b, "d_lora_b", parts * n_out * r, bf)
+    _on_cuda(x=x, w=w, dy=dy, dx=dx, lora_a=lora_a, lora_b=lora_b, d_lora_a=d_lora_a, d_lora_b=d_lora_b)
+    _workspace(workspace)
+    _check("lora_proj_bwd", capi().lora_proj_bwd(
+        _ptr(x), _ptr(w), _ptr(lora_a), _ptr(lora_b), _ptr(dy), _ptr(dx), _ptr(d_lora_a), _ptr(d_lora_b),
+        T, K, n_out, parts, r, float(scaling), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
 
 
 def get_device_error():

@@ -90,6 +90,26 @@ cudaError_t launch_lora_proj(const CUtensorMap& tx, const CUtensorMap& tw, const
                              int rope_parts, int head_dim, int seq_len, const float* cos_tab, const float* sin_tab,
                              int n_sm, int* err, cudaStream_t st);
 
+// Backward of the projections (lora_bwd_sm100.cu): g = bf16(s dy_p b_pad_p) [parts, T, 64], then
+// dx = sum_p dy_p W_p + g_p a_pad_p, dA_acc += g^T x and dB_acc += dy_p^T u_p (fp32, zeroed here),
+// then dA, dB in bf16.  Tensor maps (3-D, 128-byte swizzle, 64-column boxes):
+//   dy_k {n_out, T, parts} 128-row boxes; dy_mn, bpad {64, n_out, parts}, w_mn {K, n_out, parts},
+//   apad {K, 64, parts}, g_mn / u_mn {64, T, parts}, x_mn {K, T, 1}: 64-row boxes; g_k {64, T, parts} 128-row.
+cudaError_t launch_lora_bwd(const CUtensorMap& dy_k, const CUtensorMap& dy_mn, const CUtensorMap& bpad,
+                            const CUtensorMap& w_mn, const CUtensorMap& g_k, const CUtensorMap& apad,
+                            const CUtensorMap& g_mn, const CUtensorMap& x_mn, const CUtensorMap& u_mn, void* g,
+                            void* dx, float* da_acc, float* db_acc, void* da, void* db, int T, int K, int n_out,
+                            int parts, int r, float scaling, int n_sm, int* err, cudaStream_t st);
+
+// Halo rows of the sequence-sharded path (s2attn_halo.cu): rows [0, G/2) of heads
+// [H - shift_heads, H) of up to kHaloMaxTensors tensors, to (to_buf = 1) or from (0)
+// contiguous buffers [B, G/2, shift_heads, D] (bf16 rows) or [B, shift_heads, G/2] (fp32 lse).
+constexpr int kHaloMaxTensors = 8;
+cudaError_t launch_halo_rows(void* const* x, void* const* buf, int n, int to_buf, int B, int N, int H, int D,
+                             int G, int shift_heads, int n_sm, cudaStream_t st);
+cudaError_t launch_halo_lse(float* const* x, float* const* buf, int n, int to_buf, int B, int N, int H, int G,
+                            int shift_heads, int n_sm, cudaStream_t st);
+
 // RoPE-PI in place on bf16 q and k, with a cos/sin table [N, D/2] (fp32 each).
 cudaError_t launch_rope_pi(void* q, void* k, const float* cos_tab, const float* sin_tab, int B, int N, int H,
                            int D, cudaStream_t st);

@@ -323,6 +323,35 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
   return cuda_status(s2::launch_dq_convert(dq_acc, dq, s, st));
 }
 
+int s2attn_halo_rows(void* const* x, void* const* buf, int n_tensors, int to_buf, int B, int N, int H, int D,
+                     int G, int shift_heads, void* stream) {
+  int rc = check_shape(B, N, H, D, G, shift_heads);
+  if (rc) return rc;
+  if (shift_heads < 1 || n_tensors < 1 || n_tensors > s2::kHaloMaxTensors || !x || !buf) return S2ATTN_ERR_INVALID_ARG;
+  if ((D * 2) % 16 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  for (int i = 0; i < n_tensors; ++i)
+    if (!aligned16(x[i]) || !aligned16(buf[i])) return S2ATTN_ERR_INVALID_ARG;
+  const int n_sm = sm_count();
+  if (n_sm <= 0) return S2ATTN_ERR_CUDA;
+  return cuda_status(s2::launch_halo_rows(x, buf, n_tensors, to_buf ? 1 : 0, B, N, H, D, G, shift_heads, n_sm,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int s2attn_halo_lse(float* const* lse, float* const* buf, int n_tensors, int to_buf, int B, int N, int H, int G,
+                    int shift_heads, void* stream) {
+  int rc = check_shape(B, N, H, 1, G, shift_heads);
+  if (rc) return rc;
+  if (shift_heads < 1 || n_tensors < 1 || n_tensors > s2::kHaloMaxTensors || !lse || !buf)
+    return S2ATTN_ERR_INVALID_ARG;
+  for (int i = 0; i < n_tensors; ++i)
+    if (!lse[i] || !buf[i] || (reinterpret_cast<uintptr_t>(lse[i]) & 3u) || (reinterpret_cast<uintptr_t>(buf[i]) & 3u))
+      return S2ATTN_ERR_INVALID_ARG;
+  const int n_sm = sm_count();
+  if (n_sm <= 0) return S2ATTN_ERR_CUDA;
+  return cuda_status(s2::launch_halo_lse(lse, buf, n_tensors, to_buf ? 1 : 0, B, N, H, G, shift_heads, n_sm,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 size_t s2attn_decode_workspace_bytes(int B, int M, int N, int H, int D) {
   if (check_decode_shape(B, M, N, H, D)) return 0;
   return decode_part_o_bytes(B, M, N, H, D) +
@@ -490,6 +519,63 @@ int lora_proj_fwd(const void* x, const void* w, const void* lora_a, const void* 
   }
   return cuda_status(s2::launch_lora_proj(tx, tw, tu, tb, y, T, K, n_out, parts, r, rope_parts, head_dim, seq_len,
                                           tab.cos_d, tab.sin_d, sm_count(), err, st));
+}
+
+size_t lora_proj_bwd_workspace_bytes(int T, int K, int n_out, int parts, int r) {
+  if (T < 1 || K < 1 || n_out < 1 || parts < 1 || r < 0 || r > s2::kLoraMaxRank) return 0;
+  const size_t apad = align256((size_t)parts * s2::kLoraRankPad * K * 2);
+  const size_t bpad = align256((size_t)parts * n_out * s2::kLoraRankPad * 2);
+  const size_t da_acc = align256((size_t)((parts * s2::kLoraRankPad + 127) / 128) * 128 * K * 4);
+  const size_t db_acc = align256((size_t)parts * n_out * s2::kLoraRankPad * 4);
+  return 2 * lora_u_bytes(T, parts) + apad + bpad + da_acc + db_acc;   // u, g, a_pad, b_pad, accumulators
+}
+
+int lora_proj_bwd(const void* x, const void* w, const void* lora_a, const void* lora_b, const void* dy, void* dx,
+                  void* d_lora_a, void* d_lora_b, int T, int K, int n_out, int parts, int r, float scaling,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 1 || K < 8 || K % 8 != 0 || n_out < 1 || parts < 1 || r < 0 || r > s2::kLoraMaxRank)
+    return S2ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(dy) || !aligned16(dx)) return S2ATTN_ERR_INVALID_ARG;
+  if (r > 0 && (!aligned16(lora_a) || !lora_b || !d_lora_a || !d_lora_b || !std::isfinite(scaling)))
+    return S2ATTN_ERR_INVALID_ARG;
+  if (n_out % s2::kLoraProjTileN != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if (K < 64) return S2ATTN_ERR_UNSUPPORTED;   // the tensor maps' 64-column boxes must fit in a row of x and W
+  if ((long long)parts * n_out > INT_MAX || (long long)T + 128 > INT_MAX) return S2ATTN_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return S2ATTN_ERR_WORKSPACE;
+  if (workspace_bytes < lora_proj_bwd_workspace_bytes(T, K, n_out, parts, r)) return S2ATTN_ERR_WORKSPACE;
+  int* err = error_word_ptr();
+  if (!err) return S2ATTN_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const size_t ub = lora_u_bytes(T, parts);
+  void* u = ws;
+  void* g = ws + ub;
+  void* a_pad = ws + 2 * ub;
+  void* b_pad = static_cast<char*>(a_pad) + align256((size_t)parts * s2::kLoraRankPad * K * 2);
+  float* da_acc = reinterpret_cast<float*>(static_cast<char*>(b_pad) +
+                                           align256((size_t)parts * n_out * s2::kLoraRankPad * 2));
+  float* db_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(da_acc) +
+                                           align256((size_t)((parts * s2::kLoraRankPad + 127) / 128) * 128 * K * 4));
+  const int RP = s2::kLoraRankPad;
+  CUtensorMap dy_k, dy_mn, bpad, w_mn, g_k, apad, g_mn, x_mn, u_mn, tx, ta;
+  bool ok = map_rows_bf16(&dy_k, dy, 3, n_out, T, parts, 64, 128) && map_rows_bf16(&dy_mn, dy, 3, n_out, T, parts, 64, 64) &&
+            map_rows_bf16(&w_mn, w, 3, K, n_out, parts, 64, 64) && map_rows_bf16(&x_mn, x, 3, K, T, 1, 64, 64);
+  if (r > 0)
+    ok = ok && map_rows_bf16(&bpad, b_pad, 3, RP, n_out, parts, 64, 64) && map_rows_bf16(&g_k, g, 3, RP, T, parts, 64, 128) &&
+         map_rows_bf16(&apad, a_pad, 3, K, RP, parts, 64, 64) && map_rows_bf16(&g_mn, g, 3, RP, T, parts, 64, 64) &&
+         map_rows_bf16(&u_mn, u, 3, RP, T, parts, 64, 64) && map_rows_bf16(&tx, x, 2, K, T, 1, 64, 128) &&
+         map_rows_bf16(&ta, a_pad, 2, K, (uint64_t)parts * RP, 1, 64, RP);
+  else
+    bpad = g_k = apad = g_mn = u_mn = dy_k;   // unused without an adapter
+  if (!ok) return S2ATTN_ERR_CUDA;
+  cudaError_t e = cudaSuccess;
+  if (r > 0) {
+    e = s2::launch_lora_pad(lora_a, lora_b, a_pad, b_pad, parts, r, K, n_out, st);
+    if (e == cudaSuccess) e = s2::launch_lora_down(tx, ta, u, T, K, parts, scaling, sm_count(), err, st);
+    if (e != cudaSuccess) return S2ATTN_ERR_CUDA;
+  }
+  return cuda_status(s2::launch_lora_bwd(dy_k, dy_mn, bpad, w_mn, g_k, apad, g_mn, x_mn, u_mn, g, dx, da_acc, db_acc,
+                                         d_lora_a, d_lora_b, T, K, n_out, parts, r, scaling, sm_count(), err, st));
 }
 
 int s2attn_selftest_bounded_wait(unsigned timeout_us, void* stream) {

@@ -8,23 +8,34 @@ starting at p * Np (Np a multiple of G):
   * the rolled groups of a shifted head start G/2 tokens into each run, so the last one
     of rank p ends G/2 tokens into rank p+1's run, and rank P-1's wraps round to rank 0's
     (the roll is cyclic).
-Each rank therefore receives the first G/2 rows of the next rank (shifted heads only),
-runs the kernels on a local tensor whose shifted heads hold its rows [G/2, Np) followed
-by that halo -- so every rolled group is a plain group of the local tensor, computed
-with shift_heads = 0 -- and sends the results of the halo rows back to their owner.
+
+The library's kernels roll a shifted head cyclically inside the tensors they are given:
+on a rank's own run their last rolled group reads the run's tail followed by the run's
+rows [0, G/2).  Those rows of the shifted heads are exactly what this rank does not need
+(they belong to the previous rank's last group), and the next rank's first G/2 rows (the
+halo) are exactly what it lacks.  So each call
+  1. copies its rows [0, G/2) of the shifted heads out (halo_rows), sends them to the
+     previous rank and receives the next rank's (exchange),
+  2. writes the received halo into those rows (put_halo_rows) and runs the unmodified
+     kernels with the shift, then writes its own rows back,
+  3. copies the results that landed in rows [0, G/2) -- the halo tokens' results -- out,
+     sends them to the next rank (their owner) and writes the ones it receives from the
+     previous rank into its own rows.
+Only G/2 rows of the shifted heads per tensor are copied or sent; no local copy of a whole
+tensor is made.  The copies are this library's halo kernels (s2attn_halo_rows and
+s2attn_halo_lse), the exchange is torch.distributed point-to-point (NCCL over NVLink
+between GPUs; gloo on CPU), received into this rank's memory before a kernel reads it.
 Tokens belong to exactly one group per head, so results are moved, never summed.
 
-The exchanges are point-to-point sends and receives between ring neighbours through
-torch.distributed (NCCL over NVLink between GPUs; gloo on CPU).  A halo of G/2 rows is
-copied into this rank's memory before any kernel reads it.  The steps are public:
-to_local (exchange and local layout), the kernels with shift_heads = 0, and to_owner
-(un-roll and return of the halo rows); sharded_fwd / sharded_bwd compose them with this
-library's CUDA kernels.
+sharded_fwd and sharded_bwd modify the caller's input tensors (rows [0, G/2) of the
+shifted heads) while they run and restore them before they return, on the current
+stream: other streams must not read those tensors meanwhile.
 """
 import torch
 import torch.distributed as dist
 
-__all__ = ["shard_range", "to_local", "to_owner", "sharded_fwd", "sharded_bwd"]
+__all__ = ["shard_range", "exchange", "halo_rows", "put_halo_rows", "halo_lse", "put_halo_lse",
+           "sharded_fwd", "sharded_bwd"]
 
 
 def shard_range(N, G, world, rank):
@@ -43,7 +54,7 @@ def _world(group):
     return 1, 0
 
 
-def _ring_shift(tensors, step, group):
+def exchange(tensors, step, group=None):
     """Sends each tensor to rank (r + step) mod P and returns the tensors received from
     rank (r - step) mod P (same shapes and dtypes).  With one rank the tensors come back."""
     world, rank = _world(group)
@@ -61,6 +72,65 @@ def _ring_shift(tensors, step, group):
     return recvs
 
 
+# ---- the four primitives: the halo copies (library kernels) and the attention calls -----
+
+def _rows_copy(xs, bufs, to_buf, G, shift_heads):
+    from . import s2attn_halo_rows
+    s2attn_halo_rows(list(xs), list(bufs), to_buf, G, shift_heads)
+
+
+def _lse_copy(lses, bufs, to_buf, G, shift_heads):
+    from . import s2attn_halo_lse
+    s2attn_halo_lse(list(lses), list(bufs), to_buf, G, shift_heads)
+
+
+def _attn_fwd(q, k, v, G, shift_heads):
+    from . import s2attn_fwd
+    B, N, H, D = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    s2attn_fwd(q, k, v, o, lse, G, shift_heads)
+    return o, lse
+
+
+def _attn_bwd(q, k, v, o, dout, lse, G, shift_heads):
+    from . import s2attn_bwd, s2attn_bwd_workspace_bytes
+    B, N, H, D = q.shape
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(s2attn_bwd_workspace_bytes(B, N, H, D), dtype=torch.uint8, device=q.device)
+    s2attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, G, shift_heads, ws)
+    return dq, dk, dv
+
+
+# ---- the halo steps --------------------------------------------------------------------
+
+def halo_rows(xs, G, shift_heads):
+    """Rows [0, G/2) of the shifted heads of each [B, Np, H, D] tensor in xs, as new
+    contiguous [B, G/2, shift_heads, D] tensors (one library launch)."""
+    B, Np, H, D = xs[0].shape
+    bufs = [torch.empty((B, G // 2, shift_heads, D), dtype=x.dtype, device=x.device) for x in xs]
+    _rows_copy(xs, bufs, True, G, shift_heads)
+    return bufs
+
+
+def put_halo_rows(bufs, xs, G, shift_heads):
+    """Writes each [B, G/2, shift_heads, D] buffer into rows [0, G/2) of the shifted heads of
+    the matching tensor in xs (one library launch)."""
+    _rows_copy(xs, bufs, False, G, shift_heads)
+
+
+def halo_lse(lses, G, shift_heads):
+    """The same rows of [B, H, Np] fp32 statistics, as new [B, shift_heads, G/2] tensors."""
+    B, H, Np = lses[0].shape
+    bufs = [torch.empty((B, shift_heads, G // 2), dtype=x.dtype, device=x.device) for x in lses]
+    _lse_copy(lses, bufs, True, G, shift_heads)
+    return bufs
+
+
+def put_halo_lse(bufs, lses, G, shift_heads):
+    _lse_copy(lses, bufs, False, G, shift_heads)
+
+
 def _check(x, G, shift_heads):
     B, Np, H, D = x.shape
     if Np % G or shift_heads < 0 or shift_heads > H or (shift_heads and G % 2):
@@ -68,112 +138,46 @@ def _check(x, G, shift_heads):
     return B, Np, H, D
 
 
-def _to_local(xs, halos, G, hs):
-    """The local tensors: shifted heads (index >= hs) hold rows [G/2, Np) then the halo."""
-    half = G // 2
-    out = []
-    for x, halo in zip(xs, halos):
-        z = x.clone()
-        z[:, : x.shape[1] - half, hs:] = x[:, half:, hs:]
-        z[:, x.shape[1] - half:, hs:] = halo
-        out.append(z)
-    return out
-
-
-def _lse_to_local(lse, halo, G, hs):
-    half = G // 2
-    z = lse.clone()
-    z[:, hs:, : lse.shape[2] - half] = lse[:, hs:, half:]
-    z[:, hs:, lse.shape[2] - half:] = halo
-    return z
-
-
-def _from_local(zs, G, hs, group):
-    """Undoes _to_local: local rows [0, Np - G/2) of the shifted heads go back to tokens
-    [G/2, Np), and the halo rows' results go to the next rank, which owns those tokens."""
-    half = G // 2
-    tails = [z[:, z.shape[1] - half:, hs:] for z in zs]
-    heads = _ring_shift(tails, +1, group)
-    out = []
-    for z, head in zip(zs, heads):
-        x = z.clone()
-        x[:, half:, hs:] = z[:, : z.shape[1] - half, hs:]
-        x[:, :half, hs:] = head
-        out.append(x)
-    return out
-
-
-def _lse_from_local(lse_z, G, hs, group):
-    half = G // 2
-    (head,) = _ring_shift([lse_z[:, hs:, lse_z.shape[2] - half:]], +1, group)
-    x = lse_z.clone()
-    x[:, hs:, half:] = lse_z[:, hs:, : lse_z.shape[2] - half]
-    x[:, hs:, :half] = head
-    return x
-
-
-def to_local(xs, G, shift_heads, group=None, lse=None):
-    """The local layout of this rank's inputs: the shifted heads of each [B, Np, H, D] tensor
-    in `xs` hold rows [G/2, Np) followed by the next rank's first G/2 rows, exchanged here;
-    the other heads are unchanged.  With `lse` ([B, H, Np]) its shifted heads are laid out
-    the same way.  Returns the list of local tensors (and the local lse when given)."""
-    B, Np, H, D = _check(xs[0], G, shift_heads)
-    hs, half = H - shift_heads, G // 2
-    if shift_heads == 0:
-        return (list(xs), lse) if lse is not None else list(xs)
-    sends = [x[:, :half, hs:] for x in xs] + ([lse[:, hs:, :half]] if lse is not None else [])
-    halos = _ring_shift(sends, -1, group)
-    zs = _to_local(xs, halos[: len(xs)], G, hs)
-    if lse is None:
-        return zs
-    return zs, _lse_to_local(lse, halos[len(xs)], G, hs)
-
-
-def to_owner(zs, G, shift_heads, group=None, lse=None):
-    """Undoes to_local for results computed on the local layout: each tensor's shifted heads
-    go back to this rank's rows, and the halo rows' results travel to the next rank, which
-    owns those tokens.  Returns the list of tensors (and the lse when given)."""
-    H = zs[0].shape[2]
-    hs = H - shift_heads
-    if shift_heads == 0:
-        return (list(zs), lse) if lse is not None else list(zs)
-    out = _from_local(list(zs), G, hs, group)
-    if lse is None:
-        return out
-    return out, _lse_from_local(lse, G, hs, group)
-
-
-def _cuda_fwd(q, k, v, G):
-    from . import s2attn_fwd
-    B, N, H, D = q.shape
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    s2attn_fwd(q, k, v, o, lse, G, 0)
-    return o, lse
-
-
-def _cuda_bwd(q, k, v, o, dout, lse, G):
-    from . import s2attn_bwd, s2attn_bwd_workspace_bytes
-    B, N, H, D = q.shape
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    ws = torch.empty(s2attn_bwd_workspace_bytes(B, N, H, D), dtype=torch.uint8, device=q.device)
-    s2attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, G, 0, ws)
-    return dq, dk, dv
-
-
 def sharded_fwd(q, k, v, G, shift_heads, group=None):
     """S^2-Attn forward on this rank's run of tokens ([B, Np, H, D] bf16 CUDA tensors).
     Returns this rank's o [B, Np, H, D] and lse [B, H, Np], equal to the rows [t0, t1) of
-    the unsharded call (shard_range gives t0, t1)."""
-    qz, kz, vz = to_local((q, k, v), G, shift_heads, group)
-    oz, lse_z = _cuda_fwd(qz, kz, vz, G)
-    (o,), lse = to_owner([oz], G, shift_heads, group, lse=lse_z)
+    the unsharded call (shard_range gives t0, t1).  q, k, v are restored before returning."""
+    _check(q, G, shift_heads)
+    if shift_heads == 0:
+        return _attn_fwd(q, k, v, G, 0)
+    xs = [q, k, v]
+    own = halo_rows(xs, G, shift_heads)
+    halo = exchange(own, -1, group)              # the next rank's first G/2 rows
+    put_halo_rows(halo, xs, G, shift_heads)
+    try:
+        o, lse = _attn_fwd(q, k, v, G, shift_heads)
+    finally:
+        put_halo_rows(own, xs, G, shift_heads)   # q, k, v as the caller gave them
+    # rows [0, G/2) of o and lse hold the halo tokens' results: to their owner, the next rank
+    res = halo_rows([o], G, shift_heads) + halo_lse([lse], G, shift_heads)
+    back = exchange(res, +1, group)
+    put_halo_rows(back[:1], [o], G, shift_heads)
+    put_halo_lse(back[1:], [lse], G, shift_heads)
     return o, lse
 
 
 def sharded_bwd(q, k, v, o, dout, lse, G, shift_heads, group=None):
     """S^2-Attn backward on this rank's run of tokens: dq, dk, dv [B, Np, H, D], equal to
-    the rows [t0, t1) of the unsharded backward."""
-    (qz, kz, vz, oz, dz), lse_z = to_local((q, k, v, o, dout), G, shift_heads, group, lse=lse)
-    dqz, dkz, dvz = _cuda_bwd(qz, kz, vz, oz, dz, lse_z, G)
-    return tuple(to_owner([dqz, dkz, dvz], G, shift_heads, group))
+    the rows [t0, t1) of the unsharded backward.  q, k, v, o, dout, lse are restored."""
+    _check(q, G, shift_heads)
+    if shift_heads == 0:
+        return _attn_bwd(q, k, v, o, dout, lse, G, 0)
+    xs = [q, k, v, o, dout]
+    own = halo_rows(xs, G, shift_heads)
+    own_lse = halo_lse([lse], G, shift_heads)
+    got = exchange(own + own_lse, -1, group)
+    put_halo_rows(got[:len(xs)], xs, G, shift_heads)
+    put_halo_lse(got[len(xs):], [lse], G, shift_heads)
+    try:
+        dq, dk, dv = _attn_bwd(q, k, v, o, dout, lse, G, shift_heads)
+    finally:
+        put_halo_rows(own, xs, G, shift_heads)
+        put_halo_lse(own_lse, [lse], G, shift_heads)
+    back = exchange(halo_rows([dq, dk, dv], G, shift_heads), +1, group)
+    put_halo_rows(back, [dq, dk, dv], G, shift_heads)
+    return dq, dk, dv

@@ -1,9 +1,11 @@
-"""Sequence-sharded S^2-Attn on CPU: gloo ranks exchange the G/2 halos of the shifted heads
-(to_local), the test runs the fp64 oracle with shift_heads = 0 on each rank's local layout,
-and the results go back to their owners (to_owner); the rows, put side by side, must equal
+"""Sequence-sharded S^2-Attn on CPU: gloo ranks run the library's sharded_fwd / sharded_bwd
+with their four device primitives replaced by CPU stand-ins that this test defines -- the
+halo copies by tensor slicing and the attention calls by the fp64 oracle with the shift.
+The exchange steps (which rows go to which rank, in which direction, and the restore of
+the inputs) are the library's own.  The rows of all ranks, put side by side, must equal
 the oracle on the whole sequence with the shift -- forward (o, lse) and backward (dq, dk,
-dv).  The library's sharded_fwd / sharded_bwd compose the same steps with the CUDA kernels
-(tests/test_gpu_sharded.py)."""
+dv) -- and every input must come back unchanged.  tests/test_gpu_sharded.py runs the same
+steps with the CUDA kernels."""
 import os
 import socket
 
@@ -28,22 +30,51 @@ def _inputs(N):
     return [rng.standard_normal((B, N, H, D)) for _ in range(4)]
 
 
+def _cpu_primitives(sharded):
+    """CPU stand-ins for the halo copies (slicing) and the attention calls (the oracle)."""
+    import oracle
+
+    def rows_copy(xs, bufs, to_buf, G_, sh):
+        for x, b in zip(xs, bufs):
+            hs = x.shape[2] - sh
+            if to_buf:
+                b.copy_(x[:, : G_ // 2, hs:])
+            else:
+                x[:, : G_ // 2, hs:] = b
+
+    def lse_copy(lses, bufs, to_buf, G_, sh):
+        for x, b in zip(lses, bufs):
+            hs = x.shape[1] - sh
+            if to_buf:
+                b.copy_(x[:, hs:, : G_ // 2])
+            else:
+                x[:, hs:, : G_ // 2] = b
+
+    def attn_fwd(q, k, v, G_, sh):
+        return tuple(torch.from_numpy(a) for a in oracle.s2attn_fwd(q.numpy(), k.numpy(), v.numpy(), G_, sh))
+
+    def attn_bwd(q, k, v, o, dout, lse, G_, sh):
+        return tuple(torch.from_numpy(a) for a in oracle.s2attn_bwd(q.numpy(), k.numpy(), v.numpy(), dout.numpy(),
+                                                                     G_, sh))
+
+    sharded._rows_copy, sharded._lse_copy = rows_copy, lse_copy
+    sharded._attn_fwd, sharded._attn_bwd = attn_fwd, attn_bwd
+
+
 def _run_rank(rank, world, N):
     import sys
     sys.path.insert(0, ROOT)
-    import oracle
-    from shifted_sparse_attention_s2attn_b200.sharded import shard_range, to_local, to_owner
-    t0, t1 = shard_range(N, G, world, rank)
+    from shifted_sparse_attention_s2attn_b200 import sharded
+    _cpu_primitives(sharded)
+    t0, t1 = sharded.shard_range(N, G, world, rank)
     q, k, v, do = (torch.from_numpy(x[:, t0:t1].copy()) for x in _inputs(N))
-    # forward: local layout, oracle with shift 0, results back to their owners
-    qz, kz, vz = to_local((q, k, v), G, SH)
-    oz, lse_z = (torch.from_numpy(a) for a in oracle.s2attn_fwd(qz.numpy(), kz.numpy(), vz.numpy(), G, 0))
-    (o,), lse = to_owner([oz], G, SH, lse=lse_z)
-    # backward: o and lse travel through the exchange too; they must come back as the local layout's
-    (qz2, kz2, vz2, oz2, dz), lse_z2 = to_local((q, k, v, o, do), G, SH, lse=lse)
-    assert torch.equal(oz2, oz) and torch.equal(lse_z2, lse_z)
-    grads = oracle.s2attn_bwd(qz2.numpy(), kz2.numpy(), vz2.numpy(), dz.numpy(), G, 0)
-    dq, dk, dv = to_owner([torch.from_numpy(a) for a in grads], G, SH)
+    before = [x.clone() for x in (q, k, v, do)]
+    o, lse = sharded.sharded_fwd(q, k, v, G, SH)
+    o_in, lse_in = o.clone(), lse.clone()
+    dq, dk, dv = sharded.sharded_bwd(q, k, v, o, do, lse, G, SH)
+    # every input comes back as it was given (the halo rows are swapped back)
+    for a, b in zip((q, k, v, do, o, lse), before + [o_in, lse_in]):
+        assert torch.equal(a, b)
     return [x.numpy() for x in (o, lse, dq, dk, dv)]
 
 
