@@ -189,7 +189,8 @@ __global__ void __launch_bounds__(NTHREADS, BN <= 64 ? 2 : 1)
       ok = wait_bounded(&acc_empty[buf], ((lt >> 1) & 1) ^ 1, abort_flag, p.err);
       if (!ok) break;
       tc_fence_after();
-      for (int kb = 0; kb < n_kb_total; ++kb) {
+      // the K loop: four K=16 MMAs per stage, a compile-time count (unrolled) ...
+      for (int kb = 0; kb < p.n_kb; ++kb) {
         const int s = g % STAGES;
         ok = wait_bounded(&full[s], (g / STAGES) & 1, abort_flag, p.err);
         if (!ok) break;
@@ -197,11 +198,24 @@ __global__ void __launch_bounds__(NTHREADS, BN <= 64 ? 2 : 1)
         const uint32_t sa = s_base + s * C::STAGE_BYTES, sb = sa + C::A_BYTES;
         // K-major operands: 128-byte rows, 8-row groups 1024 B apart; K=16 steps are 32 B
         const uint64_t da = sdesc_sw128(sa, 16, 1024), db = sdesc_sw128(sb, 16, 1024);
-        const int nk = (LORA && kb == p.n_kb) ? p.lora_k16 : BK / 16;
-        for (int kk = 0; kk < nk; ++kk)
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
           mma_ss(d, sdesc_add(da, kk * 32), sdesc_add(db, kk * 32), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&empty[s]);
         ++g;
+      }
+      // ... then the rank block, ceil(r/16) MMAs
+      if (LORA && ok) {
+        const int s = g % STAGES;
+        ok = wait_bounded(&full[s], (g / STAGES) & 1, abort_flag, p.err);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t sa = s_base + s * C::STAGE_BYTES, sb = sa + C::A_BYTES;
+          const uint64_t da = sdesc_sw128(sa, 16, 1024), db = sdesc_sw128(sb, 16, 1024);
+          for (int kk = 0; kk < p.lora_k16; ++kk) mma_ss(d, sdesc_add(da, kk * 32), sdesc_add(db, kk * 32), idesc, 1u);
+          mma_commit(&empty[s]);
+          ++g;
+        }
       }
       if (!ok) break;
       mma_commit(&acc_full[buf]);
