@@ -28,8 +28,12 @@
 // pairs over columns [64w, 64w+32); dP^T [128,256), which dQ^T reuses once the dS warps have read dP^T;
 // dK [256,384); dV [384,512).
 // MMA issue order per query tile g (one thread; tcgen05 MMAs execute in issue order):
-//   dV(g) | dP(g) [after dQ(g-1) was drained] | S(g+1) | dQ(g), dK(g)
-// so S(g+1) overlaps the dS work and dK(g), dV(g+1) overlap the dQ(g) drain.
+//   dP(g) [after dQ(g-1) was drained] | dV(g) [after P(g)] | S(g+1) | dQ(g), dK(g)
+// dP(g) needs only dO(g) and the drained dP/dQ columns, so it runs while the P/dS warps
+// are still computing P(g), and dS(g) can start as soon as P(g) is done: the warps' P and
+// dS passes follow each other with no wait for a dV + dP round trip in between.  dK(g-1)
+// overlaps the dQ(g-1) drain, and S(g+1) the dS(g) work.  dS^T(g) goes into the slot of
+// dO(g), which dV(g) reads: the dS warps store it only after dV(g) has completed.
 //
 // Warp roles (512 threads; registers rebalanced with setmaxnreg, see REGS_*):
 //   warps 0-3, 4-7  P / dS, thread = key row (TMEM lane); warpgroup w takes query
@@ -62,9 +66,10 @@ constexpr uint32_t OFF_DO = OFF_Q + QSTAGES * TILE;    // [DSTAGES] tiles (dO, t
 constexpr uint32_t OFF_LSE = OFF_DO + DSTAGES * TILE;  // [QSTAGES] x lse[128] fp32
 constexpr uint32_t OFF_DELTA = OFF_LSE + QSTAGES * BQ * 4;  // [DSTAGES] x delta[128] fp32
 constexpr uint32_t OFF_BAR = OFF_DELTA + DSTAGES * BQ * 4;
-constexpr int NBARS = 24;
+constexpr int NBARS = 25;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;  // the dynamic smem base must be 1024-byte aligned
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 constexpr int NTHREADS = 512;  // warpgroups: P/dS, P/dS, dQ drain, producer + MMA (+2 idle warps)
 constexpr int WARP_DQ0 = 8, WARP_LOAD = 12, WARP_MMA = 13, WARP_CVT = 14;
 // Launch: 512 threads x 128 registers = 65536.  After setmaxnreg: P/dS warpgroups keep 128,
@@ -143,6 +148,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint64_t* dkv_empty = bars + 19;
   uint64_t* drain = bars + 20;
   uint64_t* lse_ready = bars + 21;  // [3] lse(g) of Q slot g%3 rewritten as -lse*log2(e)
+  uint64_t* dv_done = bars + 24;    // dV(g) complete: dO(g) no longer read, its slot may take dS^T(g)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
 
@@ -193,6 +199,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(dkv_empty, PDS_WARPS);
     mbar_init(drain, 1);
     for (int s = 0; s < QSTAGES; ++s) mbar_init(&lse_ready[s], 1);
+    mbar_init(dv_done, 1);
     *abort_flag = (*(volatile int*)p.err != 0) ? 1 : 0;
     fence_mbar_init();
   }
@@ -268,13 +275,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // ---------------- MMA issuer ----------------
     // Each group of 8 MMAs blocks this thread until it is nearly all dispatched, so a
     // barrier check that resolves only after the previous group leaves a bubble in the
-    // tensor pipe.  The barriers of each sync point are therefore probed (non-blocking)
+    // tensor pipe.  The barriers of the next sync point are therefore probed (non-blocking)
     // before the group ahead of it is issued; a blocking wait follows only if the probe
     // found them incomplete.  Sync points per query tile g:
-    //   A: dO(g) loaded, P^T(g) in TMEM (item start: previous dK/dV read out)  -> dV(g)
-    //   B: dQ^T(g-1) drained from the shared columns                            -> dP(g)
-    //   C: Q(g+1) loaded                                                         -> S(g+1)
-    //   D: dS^T(g) in smem                                                       -> dQ(g), dK(g)
+    //   B: dO(g) loaded, dQ^T(g-1) drained from the shared columns        -> dP(g)
+    //   A: P^T(g) in TMEM (item start: previous dK/dV read out)            -> dV(g)
+    //   C: Q(g+1) loaded                                                   -> S(g+1)
+    //   D: dS^T(g) in smem                                                 -> dQ(g), dK(g)
     const uint32_t id_kq = idesc_bf16_f32(BK, BQ, false, false);   // S^T, dP^T
     const uint32_t id_dkv = idesc_bf16_f32(BK, HD, false, true);   // dV (A = P^T in TMEM), dK (A = dS^T)
     const uint32_t id_dq = idesc_bf16_f32(HD, BQ, true, true);     // dQ^T = K^T dS^T
@@ -283,10 +290,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     auto ready_a = [&](int g, int it, int s, bool block) -> bool {
       const bool need_empty = s == 0 && it > 0;
       if (!block)
-        return mbar_test_wait(&do_full[g % DSTAGES], (g / DSTAGES) & 1) && mbar_test_wait(p_ready, g & 1) &&
-               (!need_empty || mbar_test_wait(dkv_empty, (it - 1) & 1));
-      return wait_bounded(&do_full[g % DSTAGES], (g / DSTAGES) & 1, abort_flag, p.err) &&
-             wait_bounded(p_ready, g & 1, abort_flag, p.err) &&
+        return mbar_test_wait(p_ready, g & 1) && (!need_empty || mbar_test_wait(dkv_empty, (it - 1) & 1));
+      return wait_bounded(p_ready, g & 1, abort_flag, p.err) &&
              (!need_empty || wait_bounded(dkv_empty, (it - 1) & 1, abort_flag, p.err));
     };
     bool ok = true;
@@ -300,17 +305,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tc_fence_after();
       issue_kq(tmem + TM_S, sk, sq0 + (g0 % QSTAGES) * TILE, id_kq);
       mma_commit(s_full);
-      bool pre_a = false;
       for (int s = 0; s < nsteps && ok; ++s) {
         const int g = g0 + s;
         const bool next = s + 1 < nsteps;
         const uint32_t sq = sq0 + (g % QSTAGES) * TILE;
         const uint32_t sdo = sdo0 + (g % DSTAGES) * TILE;  // dO(g), later dS^T(g)
+        // ---- B: dP^T = V dO^T, into the columns dQ^T(g-1) has left
+        ok = wait_bounded(&do_full[g % DSTAGES], (g / DSTAGES) & 1, abort_flag, p.err);
+        if (ok && g > 0) ok = wait_bounded(dq_free, (g - 1) & 1, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        const bool pre_a = ready_a(g, it, s, false);
+        issue_kq(tmem + TM_DP, sv, sdo, id_kq);
+        mma_commit(dp_full);
         // ---- A: dV += P^T dO
         if (!pre_a) ok = ready_a(g, it, s, true);
         if (!ok) break;
         tc_fence_after();
-        const bool pre_b = g == 0 || mbar_test_wait(dq_free, (g - 1) & 1);
+        const bool pre_c = !next || mbar_test_wait(&q_full[(g + 1) % QSTAGES], ((g + 1) / QSTAGES) & 1);
         {
           const uint64_t db = sdesc_sw128(sdo, BOX, 1024);
 #pragma unroll
@@ -318,15 +330,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mma_ts(tmem + TM_DV, tmem + TM_S + (kk / 4) * 64 + (kk % 4) * 8, sdesc_add(db, kk * 2048), id_dkv,
                    (s > 0 || kk > 0) ? 1u : 0u);
         }
-        // ---- B: dP(g) once dQ^T(g-1) has left the shared columns.  Always issued after
-        // dV(g): its completion (dp_full) then also means dV(g) has finished reading dO(g),
-        // whose slot the dS warps overwrite with dS^T(g).
-        if (!pre_b) ok = wait_bounded(dq_free, (g - 1) & 1, abort_flag, p.err);
-        if (!ok) break;
-        tc_fence_after();
-        const bool pre_c = !next || mbar_test_wait(&q_full[(g + 1) % QSTAGES], ((g + 1) / QSTAGES) & 1);
-        issue_kq(tmem + TM_DP, sv, sdo, id_kq);
-        mma_commit(dp_full);
+        mma_commit(dv_done);  // dO(g) read: the dS warps may overwrite its slot with dS^T(g)
         // ---- C: S(g+1): its columns held P^T(g), read by the dV MMAs above (issued first)
         bool pre_d;
         if (next) {
@@ -344,7 +348,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!pre_d) ok = wait_bounded(ds_ready, g & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
-        pre_a = next && ready_a(g + 1, it, s + 1, false);
         {
           const uint64_t dds_mn = sdesc_sw128(sdo, BOX, 1024);
 #pragma unroll
@@ -451,8 +454,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(p_ready);
 
-        // dP(g) complete => every earlier MMA (dV(g) included) is too: dO(g) is dead and
-        // its slot takes dS^T(g)
+        // dP(g) complete: dP^T(g) in TMEM (delta(g) arrived with dO(g)).  dS^T(g) goes into the
+        // slot of dO(g) once dV(g) has read it (dv_done, below)
         ok = wait_bounded(&do_full[g % DSTAGES], (g / DSTAGES) & 1, abort_flag, p.err);
         if (ok) ok = wait_bounded(dp_full, g & 1, abort_flag, p.err);
         if (!ok) break;
@@ -482,11 +485,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             pk[2 * c4] = mul_bf16x2(pp[16 * half + 2 * c4], pack_bf16x2(g01.x, g01.y));
             pk[2 * c4 + 1] = mul_bf16x2(pp[16 * half + 2 * c4 + 1], pack_bf16x2(g23.x, g23.y));
           }
+          if (half == 0) ok = wait_bounded(dv_done, g & 1, abort_flag, p.err);  // dO(g) read by dV(g)
+          if (ok) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(dsrow + (((4 * half + c) ^ (kr & 7)) * 16)) =
-                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4*>(dsrow + (((4 * half + c) ^ (kr & 7)) * 16)) =
+                  make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
         }
+        if (!ok) break;
         tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
