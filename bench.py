@@ -383,6 +383,16 @@ def run_ours(args, w):
         raise SystemExit(f"device error word set during the timed region: {detail:#x}")
 
     ms_max = max_over_ranks(ms, dev)
+    if args.step_only:
+        # profiling runs: the timed step loop and nothing after it
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": whole_job_tflops(step_flops(w), args.steps, world, ms_max),
+                              "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "ms_per_step": ms_max / args.steps, "step_only": True,
+                              "config": workload_config(w)}), flush=True)
+        return 0
 
     # ---- full causal attention (inference case: one group, no shift), forward only ----
     pairs_full = B * H * N * (N + 1) // 2
@@ -816,6 +826,8 @@ def main():
     ap.add_argument("--workload", default="llama2_7b_32k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--step-only", action="store_true",
+                    help="time the step loop and stop (no other sections, no CPU baseline): for profiler captures")
     ap.add_argument("--mode", default="replicas", choices=["replicas", "sequence", "lora", "layer"],
                     help="replicas: every rank runs the whole workload (default); sequence: the "
                          "workload's sequence is split across the ranks; lora: the layer's LoRA-adapted "
