@@ -818,6 +818,62 @@ def run_layer(args, w):
     return 0
 
 
+def run_decode(args, w):
+    """--mode decode: the decoding step of full causal attention alone (one GPU): the last M rows of q
+    as queries against all N positions of k and v at the workload's shape, M = 1, 16, 128; `warmup`
+    calls, then `steps` calls timed with CUDA events.  HBM-bound: K and V are read once per call
+    (0.54 GB at 32k, larger than L2).  value = the M = 16 call's K/V read bandwidth in GB/s."""
+    import torch
+
+    import shifted_sparse_attention_s2attn_b200 as s2
+
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    B, N, H, D = w.B, w.N, w.H, w.D
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(40)
+    k, v = (torch.randn((B, N, H, D), generator=gen, device=dev).to(torch.bfloat16) for _ in range(2))
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    s2.clear_device_error()
+    out = {}
+    for M in (1, 16, 128):
+        q = torch.randn((B, M, H, D), generator=gen, device=dev).to(torch.bfloat16)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, M), dtype=torch.float32, device=dev)
+        ws = torch.empty(s2.s2attn_decode_workspace_bytes(B, M, N, H, D), dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup):
+            s2.s2attn_decode(q, k, v, o, lse, ws, stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            s2.s2attn_decode(q, k, v, o, lse, ws, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / args.steps
+        kv_bytes = 2 * B * N * H * D * 2
+        out[f"M{M}"] = {"ms": ms, "gbs": kv_bytes / (ms / 1e3) / 1e9, "frac": kv_bytes / (ms / 1e3) / 1e9 / peak}
+        del q, o, lse, ws
+    rc, detail = s2.get_device_error()
+    if rc != 0:
+        raise SystemExit(f"device error word set during the decoding steps: {detail:#x}")
+    if rank != 0:
+        return 0
+    line = {"metric": "decoding step K/V read bandwidth, GB/s (M = 16 queries)", "value": out["M16"]["gbs"],
+            "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": out["M16"]["ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "mode": "decode",
+            "config": {"workload": f"{w.name}: the last M rows of a query tensor against all N={N} positions of k, v "
+                                   f"(H={H}, D={D}); full causal attention"},
+            "roofline": {"bound": "hbm", "peak": peak, "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs"},
+            "calls": out}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -828,10 +884,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--step-only", action="store_true",
                     help="time the step loop and stop (no other sections, no CPU baseline): for profiler captures")
-    ap.add_argument("--mode", default="replicas", choices=["replicas", "sequence", "lora", "layer"],
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "sequence", "lora", "layer", "decode"],
                     help="replicas: every rank runs the whole workload (default); sequence: the "
                          "workload's sequence is split across the ranks; lora: the layer's LoRA-adapted "
-                         "projections alone; layer: one LongLoRA attention layer training step")
+                         "projections alone; layer: one LongLoRA attention layer training step; decode: the "
+                         "decoding step of full causal attention alone")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")
@@ -846,6 +903,8 @@ def main():
         return run_lora_projections(args, w)
     if args.mode == "layer":
         return run_layer(args, w)
+    if args.mode == "decode":
+        return run_decode(args, w)
     return run_ours(args, w)
 
 
