@@ -214,6 +214,7 @@ def s2attn_halo_rows(xs, bufs, to_buf, G, shift_heads, stream=None):
     for i, (x, b) in enumerate(zip(xs, bufs)):
         _extent(x, f"x[{i}]", B * N * H * D, bf16)
         _extent(b, f"buf[{i}]", B * (G // 2) * shift_heads * D, bf16)
+    for x, b in zip(xs, bufs):
         _on_cuda(x=x, buf=b)
     _check("s2attn_halo_rows", capi().s2attn_halo_rows(_ptr_array(xs), _ptr_array(bufs), len(xs), int(bool(to_buf)),
                                                        B, N, H, D, G, shift_heads, _stream(stream)))
@@ -231,6 +232,7 @@ def s2attn_halo_lse(lses, bufs, to_buf, G, shift_heads, stream=None):
     for i, (x, b) in enumerate(zip(lses, bufs)):
         _extent(x, f"lse[{i}]", B * H * N, f32)
         _extent(b, f"buf[{i}]", B * shift_heads * (G // 2), f32)
+    for x, b in zip(lses, bufs):
         _on_cuda(lse=x, buf=b)
     _check("s2attn_halo_lse", capi().s2attn_halo_lse(_ptr_array(lses), _ptr_array(bufs), len(lses),
                                                      int(bool(to_buf)), B, N, H, G, shift_heads, _stream(stream)))

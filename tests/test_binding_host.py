@@ -87,3 +87,19 @@ def test_mismatched_extents_are_rejected_before_the_device_check():
     _extent_check_fails(s2.rope_pi_apply, a["q"], short, 0.5)
     nc = torch.zeros((1, 2, 256, 128), dtype=BF).transpose(1, 2)                                 # not contiguous
     _extent_check_fails(s2.s2attn_fwd, a["q"], nc, a["v"], a["o"], a["lse"], 128, 1)
+
+
+def test_halo_copies_check_their_buffers():
+    """The sequence-sharded path's halo copies: one [B, G/2, shift_heads, D] buffer per
+    [B,N,H,D] tensor, one [B, shift_heads, G/2] buffer per [B,H,N] lse."""
+    B, N, H, D, G, sh = 2, 1024, 4, 128, 512, 2
+    xs = [torch.zeros((B, N, H, D), dtype=BF) for _ in range(3)]
+    bufs = [torch.zeros((B, G // 2, sh, D), dtype=BF) for _ in range(3)]
+    _only_device_check_fails(s2.s2attn_halo_rows, xs, bufs, True, G, sh)
+    lse, lbuf = torch.zeros((B, H, N), dtype=F32), torch.zeros((B, sh, G // 2), dtype=F32)
+    _only_device_check_fails(s2.s2attn_halo_lse, [lse], [lbuf], False, G, sh)
+    _extent_check_fails(s2.s2attn_halo_rows, xs, bufs[:2] + [torch.zeros((B, G // 2, sh + 1, D), dtype=BF)], True, G,
+                        sh)                                                                        # buffer too big
+    _extent_check_fails(s2.s2attn_halo_lse, [lse], [lbuf[:, :1].contiguous()], True, G, sh)        # buffer too small
+    with pytest.raises(ValueError):
+        s2.s2attn_halo_rows(xs, bufs[:2], True, G, sh)                                             # unequal lists
