@@ -320,9 +320,9 @@ __global__ void __launch_bounds__(Cfg<MT>::NTHREADS, 2)
 }
 
 // o[b, m, h, :] = sum_s 2^(m_s - mx) o_s / sum_s 2^(m_s - mx) l_s ;  lse = ln2 * (mx + log2 L).
-// One CTA per (b, h, m) with CG groups of HD threads: the splits' (max, sum) pairs are loaded
-// in one parallel round, and group g sums splits g, g+CG, ... of its column d with
-// independent loads, so the step costs about two memory latencies.  Split 0 holds key 0,
+// One CTA per (b, h, m) with CG groups of HD threads: the splits' (max, sum) pairs and the
+// partial outputs (group g: splits g, g+CG, ... of its column d) are loaded in one parallel
+// round, so the step costs about one memory latency.  Split 0 holds key 0,
 // visible to every query, so mx is finite.
 constexpr int CG = 4;
 __global__ void __launch_bounds__(CG * HD) decode_combine_kernel(const float* part_o, const float* part_ml,
@@ -339,6 +339,17 @@ __global__ void __launch_bounds__(CG * HD) decode_combine_kernel(const float* pa
   // launched as a programmatic dependent of the split kernel: wait until that grid has
   // completed and its writes are visible (a no-op under ordinary stream order)
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // group grp: splits grp, grp + CG, ... (at most kDecodeMaxSplits / CG = 16) of column d.  These
+  // loads do not depend on the weights, so they go out together with the (max, sum) loads below:
+  // the two rounds of memory latency overlap.
+  const float* po = part_o + ((size_t)bh * S * M + m) * HD + d;  // split s at po[s * M * HD]
+  constexpr int PER = kDecodeMaxSplits / CG;
+  float v[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int sidx = grp + u * CG;
+    v[u] = sidx < S ? po[(size_t)sidx * M * HD] : 0.0f;
+  }
   const float* ml = part_ml + (size_t)bh * S * M * 2;
   // group 0: thread d holds split d; mx = max over splits, L = sum of weighted sums
   float ms = -INFINITY, ls = 0.0f;
@@ -361,15 +372,6 @@ __global__ void __launch_bounds__(CG * HD) decode_combine_kernel(const float* pa
   for (int off = 16; off > 0; off >>= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
   if (grp == 0 && lane == 0) red[warp][1] = y;
   __syncthreads();
-  // group grp: splits grp, grp + CG, ... (at most kDecodeMaxSplits / CG = 16), loads first
-  const float* po = part_o + ((size_t)bh * S * M + m) * HD + d;  // split s at po[s * M * HD]
-  constexpr int PER = kDecodeMaxSplits / CG;
-  float v[PER];
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int sidx = grp + u * CG;
-    v[u] = sidx < S ? po[(size_t)sidx * M * HD] : 0.0f;
-  }
   float acc = 0.0f;
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
@@ -777,7 +779,10 @@ int decode_splits_tc(int B, int N, int H, int n_sm, int* tiles_per_split) {
   const int n_tiles = (N + dtc::BN - 1) / dtc::BN;
   const long long units = (long long)B * H;
   const long long slots = 2LL * n_sm;                          // two CTAs per SM
-  const long long base_ctas = units * ((n_tiles + 15) / 16);  // about 16 tiles (1024 keys) per CTA
+  // about 32 tiles (2048 keys) per CTA: the fp32 partials grow with M times the number of splits
+  // (at 32k and M = 128, 16-tile splits write and read back 138 MB of partials against 537 MB of
+  // K/V; 32-tile splits: M = 128 0.149 -> 0.137 ms, M = 64 0.122 -> 0.118 ms, M <= 16 unchanged)
+  const long long base_ctas = units * ((n_tiles + 31) / 32);
   const long long waves = (base_ctas + slots - 1) / slots;
   long long s = (waves * slots) / units;
   if (s < 1) s = 1;
