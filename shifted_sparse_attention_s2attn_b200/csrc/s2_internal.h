@@ -22,9 +22,10 @@ struct Shape {
   int B, N, H, D, G, shift_heads;
 };
 
-// Forward, bf16, D == 128: one launch of the tcgen05 kernel.
+// Forward, bf16, D == 128: one launch of the tcgen05 kernel, a persistent grid of at most
+// n_sm CTAs (one per SM).
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                             void* o, float* lse, const Shape& s, int* err, cudaStream_t st);
+                             void* o, float* lse, const Shape& s, int n_sm, int* err, cudaStream_t st);
 
 // Backward main kernel, bf16, D == 128: dK, dV written, dQ accumulated (fp32) into dq_acc.
 // Tensor maps: 128-row boxes of 64 columns, 128-byte swizzle, for q, k, v and dout.

@@ -264,7 +264,7 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     return S2ATTN_ERR_CUDA;
   int* err = error_word_ptr();
   if (!err) return S2ATTN_ERR_CUDA;
-  return cuda_status(s2::launch_fwd_sm100(tq, tk, tv, o, lse, s, err, static_cast<cudaStream_t>(stream)));
+  return cuda_status(s2::launch_fwd_sm100(tq, tk, tv, o, lse, s, sm_count(), err, static_cast<cudaStream_t>(stream)));
 }
 
 size_t s2attn_bwd_workspace_bytes(int B, int N, int H, int D) {

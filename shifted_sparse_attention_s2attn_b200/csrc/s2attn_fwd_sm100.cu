@@ -15,9 +15,15 @@
 // Work item: (batch b, head h, group j, pair m) -> the two query tiles 2m and 2m+1 of
 // the group (128 rows each), which share every K/V tile they load.  Only the causal
 // lower triangle is visited: query tile qt needs key tiles 0..qt, and only tile qt
-// (the diagonal) is masked.  Each CTA runs two items of one group, pair m and pair
-// n_pairs-1-m, so every CTA does the same number of K/V tiles; consecutive CTAs
-// share a group, which keeps that group's K/V resident in L2.
+// (the diagonal) is masked.  Pair m costs 2m+2 K/V steps.  Two schedules:
+//   fold:  one CTA per (group, f) runs pair n_pairs-1-f and then pair f, so every CTA
+//          does the same work; consecutive CTAs share a group, which keeps that
+//          group's K/V resident in L2;
+//   snake: a persistent grid of P CTAs (one per SM) over the list of all pairs,
+//          heaviest first; in round r CTA c takes item r*P + c (r even) or
+//          r*P + P-1-c (r odd).  This evens out unequal pairs when the fold leaves a
+//          large partial last wave, but concurrent CTAs work on different groups, so
+//          it is chosen only when all of K and V fits in L2.
 //
 // Warp roles (320 threads):
 //   warps 0-3  softmax for query tile 0 (thread = row; TMEM lanes 0..127)
@@ -69,6 +75,7 @@ struct Params {
   float* lse;
   int B, N, H, G, shift_heads;
   int n_qt, n_pairs, n_groups;
+  int snake;  // 1: persistent snake schedule, 0: folded pairs (one CTA per fold)
   float sl2;  // softmax scale * log2(e)
   int* err;
 };
@@ -156,22 +163,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // ---- work items: one group (b, h, j); the heavy tile pair m0 and the light pair m1 ----
+  // ---- work items ----
+  const int n_units = p.B * p.H * p.n_groups;
+  const int n_total = p.n_pairs * n_units;
   const int n_fold = (p.n_pairs + 1) / 2;
-  const int unit = (int)(blockIdx.x / n_fold);
-  const int fi = (int)(blockIdx.x % n_fold);
-  const int j = unit % p.n_groups;
-  const int h = (unit / p.n_groups) % p.H;
-  const int b = unit / (p.n_groups * p.H);
-  int ms[2];
-  int n_items = 0;
-  ms[n_items++] = p.n_pairs - 1 - fi;
-  if (fi != p.n_pairs - 1 - fi) ms[n_items++] = fi;
-  const int shift = (h >= p.H - p.shift_heads) ? p.G / 2 : 0;
-  const int group_row0 = j * p.G;
-  // first original token of the 128-row tile `tile` of this group (tiles never wrap)
-  auto tile_token0 = [&](int tile) {
-    int t = group_row0 + tile * BM + shift;
+  struct Item {
+    int m, b, h, shift, row0;  // pair, batch, head, roll, first rolled row of the group
+  };
+  // this CTA's item r, or m = -1 past its last item
+  const int cta = (int)blockIdx.x;
+  auto item_of = [&](int r) {
+    Item w;
+    w.m = -1;
+    int unit;
+    if (p.snake) {
+      const int P = (int)gridDim.x;
+      const long long i = (long long)r * P + ((r & 1) ? P - 1 - cta : cta);
+      if (i >= n_total) return w;
+      unit = (int)(i % n_units);
+      w.m = p.n_pairs - 1 - (int)(i / n_units);
+    } else {
+      const int fi = cta % n_fold;
+      unit = cta / n_fold;
+      if (r > 1 || (r == 1 && fi == p.n_pairs - 1 - fi)) return w;
+      w.m = r == 0 ? p.n_pairs - 1 - fi : fi;
+    }
+    const int j = unit % p.n_groups;
+    w.h = (unit / p.n_groups) % p.H;
+    w.b = unit / (p.n_groups * p.H);
+    w.shift = (w.h >= p.H - p.shift_heads) ? p.G / 2 : 0;
+    w.row0 = j * p.G;
+    return w;
+  };
+  // first original token of the 128-row tile `tile` of the item's group (tiles never wrap)
+  auto tile_token0 = [&](const Item& w, int tile) {
+    int t = w.row0 + tile * BM + w.shift;
     return t >= p.N ? t - p.N : t;
   };
 
@@ -210,10 +236,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tk);
     prefetch_tmap(&tv);
     bool ok = true;
-    const int row_base = b * p.N;
     int q_loads = 0, kv = 0, k_armed = 0, v_armed = 0;  // loads issued
-    for (int it = 0; it < n_items && ok; ++it) {
-      const int qa = 2 * ms[it], qb = qa + 1;
+    for (int it = 0; ok; ++it) {
+      const Item w = item_of(it);
+      if (w.m < 0) break;
+      const int row_base = w.b * p.N, h = w.h;
+      const int qa = 2 * w.m, qb = qa + 1;
       const bool has_b = qb < p.n_qt;
       const int nkv = (has_b ? qb : qa) + 1;
       if (it > 0) {
@@ -222,14 +250,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       mbar_arrive_expect_tx(q_full, (has_b ? 2u : 1u) * TILE_BYTES);
       for (int x = 0; x < NBOX; ++x) {
-        tma_load_3d(smem + OFF_Q0 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(qa), q_full);
-        if (has_b) tma_load_3d(smem + OFF_Q1 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(qb), q_full);
+        tma_load_3d(smem + OFF_Q0 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(w, qa), q_full);
+        if (has_b) tma_load_3d(smem + OFF_Q1 + x * BOX_BYTES, &tq, x * 64, h, row_base + tile_token0(w, qb), q_full);
       }
       ++q_loads;
       for (int t = 0; t < nkv; ++t, ++kv) {
         const int st = kv % STAGES;
         const uint32_t ph = (kv / STAGES) & 1;
-        const int row = row_base + tile_token0(t);
+        const int row = row_base + tile_token0(w, t);
         ok = wait_bounded(&k_empty[st], ph ^ 1, abort_flag, p.err);
         if (!ok) break;
         mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
@@ -265,8 +293,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int o_items[2] = {0, 0};  // items whose O_i has been produced
     int kv0 = 0;              // K/V ring position of tile 0 of the current item
     bool ok = true;
-    for (int it = 0; it < n_items && ok; ++it) {
-      const int qa = 2 * ms[it], qb = qa + 1;
+    for (int it = 0; ok; ++it) {
+      const Item w = item_of(it);
+      if (w.m < 0) break;
+      const int qa = 2 * w.m, qb = qa + 1;
       const bool has_b = qb < p.n_qt;
       const int nkv = (has_b ? qb : qa) + 1;
       const int qts[2] = {qa, qb};
@@ -323,8 +353,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint32_t s_phase = 0;
     int o_items = 0;
     bool ok = true;
-    for (int it = 0; it < n_items && ok; ++it) {
-      const int qa = 2 * ms[it], qb = qa + 1;
+    for (int it = 0; ok; ++it) {
+      const Item w = item_of(it);
+      if (w.m < 0) break;
+      const int qa = 2 * w.m, qb = qa + 1;
       const bool has_b = qb < p.n_qt;
       if (i == 1 && !has_b) continue;
       const int qt = i == 0 ? qa : qb;
@@ -385,7 +417,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (!ok) break;
       // ---- epilogue: O row / l, stored at its original token; lse in natural log ----
       tc_fence_after();
-      const int tok = tile_token0(qt) + row;
+      const int tok = tile_token0(w, qt) + row;
+      const int b = w.b, h = w.h;
       const float inv_l = 1.0f / l_run;
       const size_t o_first = ((size_t)(b * p.N + tok) * p.H + h) * HD;
       const size_t lse_idx = ((size_t)b * p.H + h) * p.N + tok;
@@ -429,7 +462,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace fwd
 
 cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
-                             float* lse, const Shape& s, int* err, cudaStream_t st) {
+                             float* lse, const Shape& s, int n_sm, int* err, cudaStream_t st) {
   fwd::Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -443,8 +476,17 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
   p.n_groups = s.N / s.G;
   p.sl2 = (float)(1.4426950408889634 / sqrt((double)s.D));
   p.err = err;
-  const long long grid = (long long)((p.n_pairs + 1) / 2) * s.B * s.H * p.n_groups;
-  if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const long long n_units = (long long)s.B * s.H * p.n_groups;
+  const long long n_items = (long long)p.n_pairs * n_units;
+  if (n_items <= 0 || n_items > 0x7fffffffLL || n_sm <= 0) return cudaErrorInvalidValue;
+  // The fold's equal CTAs run in ceil(folds / n_sm) waves; when the last wave is much
+  // less than full and K and V together fit in L2 (the snake's concurrent CTAs read
+  // different groups), the snake schedule balances the pairs instead.
+  const long long folds = (long long)((p.n_pairs + 1) / 2) * n_units;
+  const long long waves = (folds + n_sm - 1) / n_sm;
+  const double kv_bytes = 2.0 * s.B * s.N * s.H * s.D * 2;
+  p.snake = (folds * 10 < waves * n_sm * 9 && kv_bytes <= 160e6) ? 1 : 0;
+  const long long grid = p.snake ? (n_items < n_sm ? n_items : n_sm) : folds;
   cudaError_t e = cudaFuncSetAttribute(fwd::s2attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)fwd::SMEM_BYTES);
   if (e != cudaSuccess) return e;
