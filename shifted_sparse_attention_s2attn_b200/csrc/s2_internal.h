@@ -29,9 +29,10 @@ cudaError_t launch_fwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
 
 // Backward main kernel, bf16, D == 128: dK, dV written, dQ accumulated (fp32) into dq_acc.
 // Tensor maps: 128-row boxes of 64 columns, 128-byte swizzle, for q, k, v and dout.
+// n_sm: the device's SM count (short folds run on a persistent grid of one CTA per SM).
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc, void* dk,
-                             void* dv, const Shape& s, int* err, cudaStream_t st);
+                             void* dv, const Shape& s, int n_sm, int* err, cudaStream_t st);
 
 // delta[b,h,t] = sum_d dO*O (fp32) and dq_acc := 0.
 cudaError_t launch_bwd_preprocess(const void* o, const void* dout, float* delta, float* dq_acc, const Shape& s,

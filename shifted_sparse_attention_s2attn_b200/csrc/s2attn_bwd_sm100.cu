@@ -20,9 +20,11 @@
 //   dV += P^T dO (P^T from TMEM), dK += dS^T Q   (M = 128 keys, N = 128 dims)
 //   dQ^T = K^T dS^T                      (M = 128 dims,  N = 128 queries)
 // Every MMA has N = 128: a tcgen05 MMA with N = 64 takes as long as one with N = 128.
-// Each CTA runs two key tiles of one group, kt and n_kt-1-kt, so every CTA walks
-// the same number of query tiles, and consecutive CTAs share a group: its Q, dO and
-// dQ accumulator rows stay in L2.
+// Work is folded: fold (group, f) holds key tiles f and n_kt-1-f of one group, so every fold
+// walks the same number of query tiles, and consecutive folds share a group: its Q, dO and
+// dQ accumulator rows stay in L2.  One CTA per fold, or, when folds are short (G <= 2048:
+// the CTA's fixed start-up and drain then weigh most), a persistent grid of one CTA per SM
+// that takes folds blockIdx.x, blockIdx.x + gridDim.x, ... in turn.
 //
 // TMEM (512 columns): S^T [0,128), with P^T for queries [64w, 64w+64) written as bf16
 // pairs over columns [64w, 64w+32); dP^T [128,256), which dQ^T reuses once the dS warps have read dP^T;
@@ -89,6 +91,7 @@ struct Params {
   __nv_bfloat16* dv;
   int B, N, H, G, shift_heads;
   int n_groups, n_kt;
+  int persistent, n_folds;
   float scale, sl2;
   int* err;
 };
@@ -159,21 +162,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     return;
   }
 
-  // ---- work items: one group (b, h, j); key tiles kt0 (heavy) and n_kt-1-kt0 (light) ----
+  // ---- work items: fold (group, f) = key tiles f (heavy) and n_kt-1-f (light) ----
   const int n_fold = (p.n_kt + 1) / 2;
-  const int unit = (int)(blockIdx.x / n_fold);
-  const int fi = (int)(blockIdx.x % n_fold);
-  const int j = unit % p.n_groups;
-  const int h = (unit / p.n_groups) % p.H;
-  const int b = unit / (p.n_groups * p.H);
-  int kts[2];
-  int n_items = 0;
-  kts[n_items++] = fi;
-  if (fi != p.n_kt - 1 - fi) kts[n_items++] = p.n_kt - 1 - fi;
-  const int shift = (h >= p.H - p.shift_heads) ? p.G / 2 : 0;
-  const int group_row0 = j * p.G;
-  auto token_of = [&](int local_row) {  // original token of a local (rolled) row; tiles never wrap
-    int t = group_row0 + local_row + shift;
+  struct Item {
+    int kt, b, h, shift, row0;  // key tile, batch, head, roll, first rolled row of the group
+  };
+  // this CTA's item `it`, or kt = -1 past its last item (the persistent grid is used only
+  // when every fold holds two key tiles)
+  auto item_of = [&](int it) {
+    Item w;
+    w.kt = -1;
+    int f, sub;
+    if (p.persistent) {
+      f = (int)blockIdx.x + (it >> 1) * (int)gridDim.x;
+      sub = it & 1;
+      if (f >= p.n_folds) return w;
+    } else {
+      f = (int)blockIdx.x;
+      sub = it;
+      if (sub > 1) return w;
+    }
+    const int fi = f % n_fold, unit = f / n_fold;
+    if (sub == 1 && fi == p.n_kt - 1 - fi) return w;
+    w.kt = sub ? p.n_kt - 1 - fi : fi;
+    const int j = unit % p.n_groups;
+    w.h = (unit / p.n_groups) % p.H;
+    w.b = unit / (p.n_groups * p.H);
+    w.shift = (w.h >= p.H - p.shift_heads) ? p.G / 2 : 0;
+    w.row0 = j * p.G;
+    return w;
+  };
+  // original token of a local (rolled) row of the item's group; tiles never wrap
+  auto token_of = [&](const Item& w, int local_row) {
+    int t = w.row0 + local_row + w.shift;
     return t >= p.N ? t - p.N : t;
   };
   auto steps_of = [&](int kt) { return p.n_kt - kt; };  // query tiles kt .. n_kt-1
@@ -224,16 +245,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tv);
     prefetch_tmap(&tdo);
     bool ok = true;
-    const int row_base = b * p.N;
-    const size_t stat_base = ((size_t)b * p.H + h) * p.N;
     int kv_loads = 0, q_armed = 0, do_armed = 0;
-    for (int it = 0; it < n_items && ok; ++it) {
-      const int kt = kts[it];
+    for (int it = 0; ok; ++it) {
+      const Item w = item_of(it);
+      if (w.kt < 0) break;
+      const int kt = w.kt, h = w.h;
+      const int row_base = w.b * p.N;
+      const size_t stat_base = ((size_t)w.b * p.H + w.h) * p.N;
       if (it > 0) {
         ok = wait_bounded(kv_empty, (it - 1) & 1, abort_flag, p.err);
         if (!ok) break;
       }
-      const int key_tok0 = token_of(kt * BK);
+      const int key_tok0 = token_of(w, kt * BK);
       mbar_arrive_expect_tx(kv_full, 2 * TILE);
       for (int x = 0; x < 2; ++x) {
         tma_load_3d(smem + OFF_K + x * BOX, &tk, x * 64, h, row_base + key_tok0, kv_full);
@@ -243,7 +266,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int nsteps = steps_of(kt);
       for (int s = 0; s < nsteps; ++s) {
         const int g = q_armed;
-        const int tok = token_of((kt + s) * BQ);
+        const int tok = token_of(w, (kt + s) * BQ);
         const int qs = g % QSTAGES, ds = g % DSTAGES;
         ok = wait_bounded(&q_empty[qs], ((g / QSTAGES) & 1) ^ 1, abort_flag, p.err);
         if (!ok) break;
@@ -296,8 +319,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     };
     bool ok = true;
     int g0 = 0;  // global index of the current item's first query tile
-    for (int it = 0; it < n_items && ok; ++it) {
-      const int nsteps = steps_of(kts[it]);
+    for (int it = 0; ok; ++it) {
+      const Item w = item_of(it);
+      if (w.kt < 0) break;
+      const int nsteps = steps_of(w.kt);
       // prologue: S(g0)
       ok = wait_bounded(kv_full, it & 1, abort_flag, p.err);
       if (ok) ok = wait_bounded(&q_full[g0 % QSTAGES], (g0 / QSTAGES) & 1, abort_flag, p.err);
@@ -381,8 +406,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // instead of recomputing the 128 products in each of 256 threads.
     bool ok = true;
     int g = 0;
-    for (int it = 0; it < n_items && ok; ++it) {
-      const int nsteps = steps_of(kts[it]);
+    for (int it = 0; ok; ++it) {
+      const Item w = item_of(it);
+      if (w.kt < 0) break;
+      const int nsteps = steps_of(w.kt);
       for (int s = 0; s < nsteps; ++s, ++g) {
         ok = wait_bounded(&q_full[g % QSTAGES], (g / QSTAGES) & 1, abort_flag, p.err);
         if (!ok) break;
@@ -412,8 +439,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const float sl2 = p.sl2;
     bool ok = true;
     int g = 0;
-    for (int it = 0; it < n_items && ok; ++it) {
-      const int kt = kts[it];
+    for (int it = 0; ok; ++it) {
+      const Item w = item_of(it);
+      if (w.kt < 0) break;
+      const int kt = w.kt;
       const int nsteps = steps_of(kt);
       for (int s = 0; s < nsteps; ++s, ++g) {
         const float* lse_s = reinterpret_cast<const float*>(smem + OFF_LSE + (g % QSTAGES) * BQ * 4) + 64 * hf;
@@ -502,8 +531,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (ok) ok = wait_bounded(mma_done, it & 1, abort_flag, p.err);
       if (!ok) break;
       tc_fence_after();
-      const int tok = token_of(kt * BK) + kr;
-      const size_t row_first = ((size_t)(b * p.N + tok) * p.H + h) * HD;
+      const int tok = token_of(w, kt * BK) + kr;
+      const size_t row_first = ((size_t)(w.b * p.N + tok) * p.H + w.h) * HD;
       const bool row_ok = in_bounds(row_first, HD, (size_t)p.B * p.N * p.H * HD, p.err, (K_BWD << 8) | SITE_PDS);
       if (hf == 0)
         store_row_bf16(lane_addr + TM_DK, p.dk + row_first, p.scale, row_ok);
@@ -526,15 +555,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
     bool ok = true;
     int g = 0;
-    for (int it = 0; it < n_items && ok; ++it) {
-      const int kt = kts[it];
+    for (int it = 0; ok; ++it) {
+      const Item w = item_of(it);
+      if (w.kt < 0) break;
+      const int kt = w.kt;
       const int nsteps = steps_of(kt);
       for (int s = 0; s < nsteps; ++s, ++g) {
         ok = wait_bounded(dq_full, g & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
         // query q of this tile -> dq_acc[b, tok0 + q, h, d]; a warp covers 32 consecutive d (128 B)
-        float* dst = p.dq_acc + ((size_t)(b * p.N + token_of((kt + s) * BQ)) * p.H + h) * HD + d;
+        float* dst = p.dq_acc + ((size_t)(w.b * p.N + token_of(w, (kt + s) * BQ)) * p.H + w.h) * HD + d;
         const size_t row_stride = (size_t)p.H * HD;
 #ifdef S2ATTN_DEBUG
         // the 128 queries of the tile: dst + q * row_stride for q < 128 (the release build keeps
@@ -585,7 +616,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tdo, const float* lse, const float* delta, float* dq_acc, void* dk,
-                             void* dv, const Shape& s, int* err, cudaStream_t st) {
+                             void* dv, const Shape& s, int n_sm, int* err, cudaStream_t st) {
   bwd::Params p;
   p.lse = lse;
   p.delta = delta;
@@ -602,8 +633,14 @@ cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
   p.scale = (float)(1.0 / sqrt((double)s.D));
   p.sl2 = (float)(1.4426950408889634 / sqrt((double)s.D));
   p.err = err;
-  const long long grid = (long long)((p.n_kt + 1) / 2) * s.B * s.H * p.n_groups;
-  if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const long long folds = (long long)((p.n_kt + 1) / 2) * s.B * s.H * p.n_groups;
+  if (folds <= 0 || folds > 0x7fffffffLL || n_sm <= 0) return cudaErrorInvalidValue;
+  // Persistent only for short folds: measured (same-run A/B) +7 % at G = 2048, N = 8k and +4.5 %
+  // at G = 2048, N = 64k; neutral at G = 8192 and 2 % slower at G = 25600, where the block
+  // scheduler's dynamic assignment of equal CTAs balances better than a fixed stride.
+  p.n_folds = (int)folds;
+  p.persistent = (p.n_kt % 2 == 0 && p.n_kt <= 16) ? 1 : 0;
+  const long long grid = p.persistent ? (folds < n_sm ? folds : n_sm) : folds;
   cudaError_t e = cudaFuncSetAttribute(bwd::s2attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bwd::SMEM_BYTES);
   if (e != cudaSuccess) return e;

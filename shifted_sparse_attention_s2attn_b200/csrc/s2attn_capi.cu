@@ -181,6 +181,8 @@ __global__ void selftest_wait_kernel(int* err, unsigned long long timeout_ns) {
     s2::report_error(err, (s2::K_SELFTEST << 8) | 1);
 }
 
+int sm_count();
+
 int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout, const float* lse,
                   const float* delta, float* dq_acc, void* dk, void* dv, const s2::Shape& s, cudaStream_t st) {
   CUtensorMap tq, tk, tv, tdo;
@@ -189,7 +191,7 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dout,
     return S2ATTN_ERR_CUDA;
   int* err = error_word_ptr();
   if (!err) return S2ATTN_ERR_CUDA;
-  return cuda_status(s2::launch_bwd_sm100(tq, tk, tv, tdo, lse, delta, dq_acc, dk, dv, s, err, st));
+  return cuda_status(s2::launch_bwd_sm100(tq, tk, tv, tdo, lse, delta, dq_acc, dk, dv, s, sm_count(), err, st));
 }
 
 // SM count of the current device, looked up once per device.
