@@ -129,6 +129,12 @@ SMALL = {
     "one_tile_groups": (1, 512, 2, 128, 0, None),
     "all_heads_shifted": (1, 512, 2, 256, 2, None),
     "one_group_shifted": (1, 512, 2, 512, 1, None),   # G = N with a shifted head: causal in half-rolled order
+    # 256 query-tile pairs on the forward's persistent snake grid (a full round, then a partial
+    # odd one) and 256 backward folds on its persistent grid (some CTAs take two folds, some one)
+    "multi_round_schedules": (1, 8192, 8, 512, 4, None),
+    # the forward's folded grid (two pairs per CTA, 288 CTAs) with the backward's persistent grid
+    # taking 576 folds
+    "fold_schedule": (1, 8192, 18, 512, 9, None),
 }
 
 
