@@ -490,8 +490,10 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// P row = exp2(s * sl2 - m) with columns c > lim masked, written as bf16 pairs over the first
-// 32 TMEM columns of the row's S buffer; returns the fp32 row sum.
+// P row = exp2(s * sl2 - m) with columns c > lim masked (MASK; without it every column is
+// visible), written as bf16 pairs over the first 32 TMEM columns of the row's S buffer; returns
+// the fp32 row sum.
+template <bool MASK>
 __device__ __forceinline__ float p_row(const uint32_t (&sr)[64], int lim, float sl2, float neg_m, uint32_t t_s) {
   const float2 scale2 = make_float2(sl2, sl2), shift2 = make_float2(neg_m, neg_m);
   float2 sp[4];
@@ -502,8 +504,10 @@ __device__ __forceinline__ float p_row(const uint32_t (&sr)[64], int lim, float 
   for (int c = 0; c < 32; ++c) {
     const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, shift2);
     float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-    p0 = 2 * c <= lim ? p0 : 0.f;
-    p1 = 2 * c + 1 <= lim ? p1 : 0.f;
+    if (MASK) {
+      p0 = 2 * c <= lim ? p0 : 0.f;
+      p1 = 2 * c + 1 <= lim ? p1 : 0.f;
+    }
     sp[c % 4].x += p0;
     sp[c % 4].y += p1;
     pk[c] = pack_bf16x2(p0, p1);
@@ -665,13 +669,22 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       uint32_t s0[64];
       tmem_ld_x64(t_s, s0);
       const int lim = last_vis - (t_begin + i * BN);  // columns c <= lim are visible (may be < 0)
+      // every column of the tile visible to all rows of the warp (all but the last tiles of
+      // the sequence): no mask compares
+      const bool full = __all_sync(0xffffffffu, lim >= BN - 1);
       float mxp[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mxp[e] = -INFINITY;
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
-        mxp[c % 8] = max3f(mxp[c % 8], 2 * c <= lim ? __uint_as_float(s0[2 * c]) : -INFINITY,
-                           2 * c + 1 <= lim ? __uint_as_float(s0[2 * c + 1]) : -INFINITY);
+        for (int c = 0; c < 32; ++c)
+          mxp[c % 8] = max3f(mxp[c % 8], __uint_as_float(s0[2 * c]), __uint_as_float(s0[2 * c + 1]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          mxp[c % 8] = max3f(mxp[c % 8], 2 * c <= lim ? __uint_as_float(s0[2 * c]) : -INFINITY,
+                             2 * c + 1 <= lim ? __uint_as_float(s0[2 * c + 1]) : -INFINITY);
+      }
       const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
                              fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
       // lazy rescale: move the running max only when it grows by more than 2^8 (a row that has
@@ -682,7 +695,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;
       if (need) m_run = m_new;
       l_run *= alpha;
-      l_run += p_row(s0, lim, sl2, -m_run, t_s);
+      l_run += full ? p_row<false>(s0, lim, sl2, -m_run, t_s) : p_row<true>(s0, lim, sl2, -m_run, t_s);
       if (rescale && i > 0) {
         // O was last written by PV(i-1): wait for it, then scale this row of O
         ok = wait_bounded(pv_done, (i - 1) & 1, abort_flag, p.err);
