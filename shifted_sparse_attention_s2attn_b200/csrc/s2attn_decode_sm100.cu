@@ -427,6 +427,23 @@ cudaError_t launch_split(const CUtensorMap& tk, const CUtensorMap& tv, const Par
 // layout as above.
 namespace dtc {
 
+// Wait of the MMA-issuing thread: polls the barrier with test_wait instead of suspending in
+// try_wait, checking the abort flags and the time limit every 1024 polls.  Here it is 1.5-2.5 %
+// faster at every M (the softmax warps' arrival is seen sooner); in the attention forward and
+// backward, whose MMA thread shares its SM sub-partition with busy warps, polling was slower.
+__device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort, const int* gerr) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((n & 1023u) == 0) {
+      if (*abort || *(const volatile int*)gerr) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
+    }
+  }
+}
+
+
 constexpr int HD = 128, BM = 128, BN = kDecodeTileKeys;  // 64 keys per tile
 constexpr uint32_t QBOX = BM * 128;           // 128 rows x 128 B (64 bf16 columns)
 constexpr uint32_t KBOX = BN * 128;           // 64 rows x 128 B
@@ -625,10 +642,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const uint32_t id_s = idesc_bf16_f32(BM, BN, false, false);
     const uint32_t id_pv = idesc_bf16_f32(BM, HD, false, true);
     const uint32_t sq = smem_u32(smem + OFF_Q), sk = smem_u32(smem + OFF_K), sv = smem_u32(smem + OFF_V);
-    bool ok = wait_bounded(q_full, 0, abort_flag, p.err);
+    bool ok = wait_spin(q_full, 0, abort_flag, p.err);
     for (int i = 0; i <= n_tiles && ok; ++i) {
       if (i < n_tiles) {
-        ok = wait_bounded(&k_full[i % KST], (i / KST) & 1, abort_flag, p.err);
+        ok = wait_spin(&k_full[i % KST], (i / KST) & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
         issue_s(tmem + (uint32_t)BN * (i & 1), sq, sk + (i % KST) * KTILE, id_s);
@@ -636,8 +653,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         mma_commit(&k_empty[i % KST]);  // K(i) read once S(i) completes
       }
       if (i > 0) {
-        ok = wait_bounded(&p_ready[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, p.err);
-        if (ok) ok = wait_bounded(&v_full[(i - 1) % VST], ((i - 1) / VST) & 1, abort_flag, p.err);
+        ok = wait_spin(&p_ready[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, p.err);
+        if (ok) ok = wait_spin(&v_full[(i - 1) % VST], ((i - 1) / VST) & 1, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
         issue_pv(tmem + TM_O, tmem + (uint32_t)BN * ((i - 1) & 1), sv + ((i - 1) % VST) * KTILE, id_pv, i == 1);
