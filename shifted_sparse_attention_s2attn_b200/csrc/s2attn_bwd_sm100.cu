@@ -22,7 +22,7 @@
 // Every MMA has N = 128: a tcgen05 MMA with N = 64 takes as long as one with N = 128.
 // Work is folded: fold (group, f) holds key tiles f and n_kt-1-f of one group, so every fold
 // walks the same number of query tiles, and consecutive folds share a group: its Q, dO and
-// dQ accumulator rows stay in L2.  One CTA per fold, or, when folds are short (G <= 2048:
+// dQ accumulator rows stay in L2.  One CTA per fold, or, when folds are short (G <= 4096:
 // the CTA's fixed start-up and drain then weigh most), a persistent grid of one CTA per SM
 // that takes folds blockIdx.x, blockIdx.x + gridDim.x, ... in turn.
 //
@@ -635,11 +635,12 @@ cudaError_t launch_bwd_sm100(const CUtensorMap& tq, const CUtensorMap& tk, const
   p.err = err;
   const long long folds = (long long)((p.n_kt + 1) / 2) * s.B * s.H * p.n_groups;
   if (folds <= 0 || folds > 0x7fffffffLL || n_sm <= 0) return cudaErrorInvalidValue;
-  // Persistent only for short folds: measured (same-run A/B) +7 % at G = 2048, N = 8k and +4.5 %
-  // at G = 2048, N = 64k; neutral at G = 8192 and 2 % slower at G = 25600, where the block
-  // scheduler's dynamic assignment of equal CTAs balances better than a fixed stride.
+  // Persistent only for short folds: measured (same-run A/B) +7 % at G = 2048, N = 8k, +4.5 % at
+  // G = 2048, N = 64k, +1.4-1.8 % at G = 4096 (N = 16k, 32k); neutral at G = 8192 and 2 % slower at
+  // G = 25600, where the block scheduler's dynamic assignment of equal CTAs balances better than a
+  // fixed stride.
   p.n_folds = (int)folds;
-  p.persistent = (p.n_kt % 2 == 0 && p.n_kt <= 16) ? 1 : 0;
+  p.persistent = (p.n_kt % 2 == 0 && p.n_kt <= 32) ? 1 : 0;
   const long long grid = p.persistent ? (folds < n_sm ? folds : n_sm) : folds;
   cudaError_t e = cudaFuncSetAttribute(bwd::s2attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)bwd::SMEM_BYTES);
